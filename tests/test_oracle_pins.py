@@ -1,0 +1,437 @@
+"""Pins of the CPU oracle against things other than itself: library routines, closed
+forms, hand-derived traces, brute force and figures printed on the pages."""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthgen
+
+BF16, FP16 = oracle.BF16, oracle.FP16
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------------------- conversions
+
+def _f32_specials():
+    vals = [0.0, -0.0, 1.0, -1.0, 65504.0, 65519.0, 65520.0, 1e-8, 6e-8, 5.96e-8, 2.98e-8,
+            3.3895314e38, 3.4e38, np.inf, -np.inf, 1.17549435e-38, 1e-40, 9.2e-41,
+            np.float32(2 ** -24), np.float32(2 ** -25), np.float32(3 * 2 ** -26)]
+    return np.array(vals, np.float32)
+
+
+def _f32_sample(n=1 << 21, seed=0):
+    rng = np.random.default_rng(seed)
+    bits = rng.integers(0, 1 << 32, n, dtype=np.uint64).astype(np.uint32)
+    x = bits.view(np.float32)
+    # exact bf16 ties: low 16 bits = 0x8000
+    ties = (rng.integers(0, 1 << 16, 20000).astype(np.uint32) << 16) | 0x8000
+    # exact fp16 ties in the normal range
+    h = rng.integers(0x0400, 0x7BFF, 20000).astype(np.uint16)
+    lo = h.view(np.float16).astype(np.float32)
+    hi = (h + 1).view(np.float16).astype(np.float32)
+    mids = ((lo.astype(np.float64) + hi) / 2).astype(np.float32)
+    return np.concatenate([x, ties.view(np.float32), mids, -mids, _f32_specials()])
+
+
+def test_f32_to_bf16_matches_torch():
+    x = _f32_sample()
+    got = oracle.f32_to_half(x, BF16)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    nan = np.isnan(x)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.all((got[nan] & 0x7F80) == 0x7F80) and np.all((got[nan] & 0x7F) != 0)
+
+
+def test_f32_to_fp16_matches_numpy():
+    x = _f32_sample(seed=1)
+    got = oracle.f32_to_half(x, FP16)
+    with np.errstate(over="ignore"):
+        ref = x.astype(np.float16).view(np.uint16)
+    nan = np.isnan(x)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.all((got[nan] & 0x7C00) == 0x7C00) and np.all((got[nan] & 0x3FF) != 0)
+
+
+def test_half_to_f32_all_patterns():
+    h = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    fb = oracle.half_to_f32(h, BF16)
+    assert np.array_equal(fb.view(np.uint32), h.astype(np.uint32) << 16)
+    fh = oracle.half_to_f32(h, FP16)
+    ref = h.view(np.float16).astype(np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(fh[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+    assert np.all(np.isnan(fh[nan]))
+
+
+# ----------------------------------------------------------------------------- reduction
+
+def _bf16(vals):
+    return torch.tensor(vals, dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_reduce_is_rank_ordered_fp32_sum():
+    # 2^24 + 1 is a tie in fp32 and rounds back to 2^24 (even), while 1 - 2^24 is exact.
+    # So the rank order and the fp32 precision of the sum show in the result:
+    #   (a, b, c) = ((2^24 + 1) - 2^24)  -> 0
+    #   (a, c, b) = ((2^24 - 2^24) + 1)  -> 1
+    #   (b, a, c) = ((1 + 2^24) - 2^24)  -> 0
+    #   (b, c, a) = ((1 - 2^24) + 2^24)  -> 1
+    # A mean, an fp64 sum or another order would give something else.
+    a, b, c = 2.0 ** 24, 1.0, -(2.0 ** 24)
+    g = [_bf16([a, a, b, b]), _bf16([b, c, a, c]), _bf16([c, b, c, a])]
+    R = oracle.reduce(g, BF16)
+    assert R.tolist() == [0.0, 1.0, 0.0, 1.0]
+
+
+def test_reduce_exact_for_dyadic_inputs():
+    # multiples of 2^-10 with small integer numerators: the fp32 sum is the exact sum
+    rng = np.random.default_rng(3)
+    W, n = 8, 4096
+    ints = rng.integers(-200, 201, (W, n))
+    grads = [_bf16((ints[r] / 1024.0).tolist()) for r in range(W)]
+    R = oracle.reduce(grads, BF16)
+    assert np.array_equal(R.astype(np.float64), ints.sum(0) / 1024.0)
+
+
+def test_partition_invariance_of_sum():
+    # replicas g/W for W in {1,2,4,8}: sums of W equal bf16 copies are exact in fp32
+    rng = np.random.default_rng(4)
+    g = rng.normal(0, 1e-3, 10000).astype(np.float32)
+    gb = torch.from_numpy(g).to(torch.bfloat16)
+    ref = None
+    for W in (1, 2, 4, 8):
+        part = (gb.float() / W).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        R = oracle.reduce([part] * W, BF16)
+        if ref is None:
+            ref = R
+        assert np.array_equal(R, ref)
+    assert np.array_equal(ref, gb.float().numpy())
+
+
+# ----------------------------------------------------------------------------- norm / clip / flags
+
+def _run_one(grads_f32_list, master, dtype=BF16, cfg=None, hp=None, st=None, bucket=1 << 40):
+    grads = [oracle.f32_to_half(np.asarray(g, np.float32), dtype) for g in grads_f32_list]
+    n = grads[0].size
+    cfg = cfg or oracle.scaler_cfg(False)
+    hp = hp or oracle.hparams()
+    st = st or oracle.state_init(cfg)
+    R = np.zeros(n, np.float32)
+    m = np.zeros(n, np.float32)
+    v = np.zeros(n, np.float32)
+    master = np.array(master, np.float32)
+    params = oracle.f32_to_half(master, dtype)
+    sc = oracle.step(grads, dtype, bucket, R, master, m, v, params, dtype, cfg, hp, st)
+    return sc, dict(R=R, master=master, m=m, v=v, params=params, state=st)
+
+
+def test_norm_constant_gradient_closed_form():
+    # W replicas of the constant a: R = W*a, S = N*(W*a)^2, norm = W*|a|*sqrt(N)/scale
+    N, W, a = 4096, 4, 0.125
+    cfg = oracle.scaler_cfg(True, init_scale_power=3)
+    sc, _ = _run_one([np.full(N, a)] * W, np.zeros(N), FP16, cfg=cfg)
+    assert sc.sumsq == N * (W * a) ** 2
+    assert sc.norm == W * a * math.sqrt(N) / 8.0
+    # split over several buckets gives the same S
+    sc2, _ = _run_one([np.full(N, a)] * W, np.zeros(N), FP16,
+                      cfg=oracle.scaler_cfg(True, init_scale_power=3), bucket=1000)
+    assert sc2.sumsq == sc.sumsq
+
+
+def test_clip_coefficient():
+    # norm 2 -> c = 1/(2 + 1e-6); norm <= 1 -> c = 1 and k = 1/scale
+    sc, _ = _run_one([np.ones(4)], np.zeros(4))
+    assert sc.norm == 2.0
+    assert sc.clip_coef == np.float32(1.0 / (2.0 + 1e-6))
+    assert sc.k == np.float32(1.0 / (2.0 + 1e-6))
+    sc, _ = _run_one([np.full(4, 0.25)], np.zeros(4))
+    assert sc.norm == 0.5 and sc.clip_coef == 1.0 and sc.k == 1.0
+    sc, _ = _run_one([np.full(4, 0.25)], np.zeros(4), hp=oracle.hparams(max_grad_norm=0.0))
+    assert sc.clip_coef == 1.0  # clipping off
+
+
+@pytest.mark.parametrize("vals", [
+    [[np.inf], [0.0]], [[-np.inf], [1.0]], [[np.nan], [0.0]], [[np.inf], [-np.inf]],
+    [[65504.0], [65504.0]],  # fp16 inputs whose fp32 sum is finite: NOT an overflow
+])
+def test_overflow_detection_and_skip(vals):
+    cfg = oracle.scaler_cfg(True, init_scale_power=16)
+    grads = [np.concatenate([np.array(v, np.float32), np.zeros(7, np.float32)]) for v in vals]
+    master = np.linspace(-1, 1, 8).astype(np.float32)
+    sc, out = _run_one(grads, master, FP16, cfg=cfg)
+    finite = all(np.isfinite(v).all() for v in vals)
+    if finite:
+        assert sc.overflow == 0 and sc.skipped == 0 and out["state"].adam_t == 1
+        return
+    assert sc.overflow == 1 and sc.skipped == 1
+    assert np.array_equal(out["master"], master)  # untouched
+    assert not out["m"].any() and not out["v"].any()
+    assert np.array_equal(out["params"], oracle.f32_to_half(master, FP16))
+    assert out["state"].adam_t == 0
+    assert out["state"].cur_hysteresis == 1  # budget spent, scale kept
+    assert sc.next_scale == 65536.0
+
+
+# ----------------------------------------------------------------------------- AdamW closed forms
+
+def test_first_step_closed_form():
+    # t = 1: m^ = g and v^ = g^2, so p1 = p0*(1 - lr*wd) - lr*g/(|g| + eps)
+    rng = np.random.default_rng(5)
+    n = 20000
+    g = rng.normal(0, 1e-3, n).astype(np.float32)
+    gb = oracle.half_to_f32(oracle.f32_to_half(g, BF16), BF16)
+    p0 = rng.normal(0, 0.02, n).astype(np.float32)
+    hp = oracle.hparams()
+    sc, out = _run_one([gb], p0, hp=hp)
+    assert sc.norm < 1.0 and sc.k == 1.0
+    lr, wd, eps = 6e-5, 0.01, 1e-8
+    g64, p64 = gb.astype(np.float64), p0.astype(np.float64)
+    ref = p64 * (1 - lr * wd) - lr * g64 / (np.abs(g64) + eps)
+    assert np.max(np.abs(out["master"] - ref) / np.maximum(np.abs(ref), 1e-3)) < 1e-6
+    np.testing.assert_allclose(out["m"], 0.1 * g64, rtol=1e-6, atol=0)
+    np.testing.assert_allclose(out["v"], 0.001 * g64 * g64, rtol=1e-5, atol=0)
+    assert out["state"].adam_t == 1
+
+
+def test_constant_gradient_bias_correction():
+    # same g every step: m_t = (1 - b1^t) g and v_t = (1 - b2^t) g^2, so m^ = g, v^ = g^2
+    # and every step moves p by -lr*g/(|g|+eps) after the decay.
+    rng = np.random.default_rng(6)
+    n = 4096
+    g = oracle.half_to_f32(oracle.f32_to_half(rng.normal(0, 1e-3, n).astype(np.float32), BF16), BF16)
+    g = g[np.abs(g) > 1e-5]
+    n = g.size
+    cfg = oracle.scaler_cfg(False)
+    hp = oracle.hparams()
+    st = oracle.state_init(cfg)
+    R = np.zeros(n, np.float32)
+    master = np.zeros(n, np.float32)
+    m = np.zeros(n, np.float32)
+    v = np.zeros(n, np.float32)
+    params = np.zeros(n, np.uint16)
+    gh = oracle.f32_to_half(g, BF16)
+    p_ref = np.zeros(n, np.float64)
+    for t in range(1, 31):
+        sc = oracle.step([gh], BF16, 1 << 40, R, master, m, v, params, BF16, cfg, hp, st)
+        mhat = m / (1 - 0.9 ** t)
+        vhat = v / (1 - 0.999 ** t)
+        np.testing.assert_allclose(mhat, g, rtol=2e-5)
+        np.testing.assert_allclose(vhat, g.astype(np.float64) ** 2, rtol=2e-5)
+        p_ref = p_ref * (1 - 6e-5 * 0.01) - 6e-5 * g / (np.abs(g) + 1e-8)
+    assert sc.adam_t == 30
+    np.testing.assert_allclose(master, p_ref, rtol=2e-5)
+
+
+def test_zero_gradient_pure_decay():
+    # g = 0: m = v = 0 and p_t = p0 * (1 - lr*wd)^t
+    p0 = np.array([0.5, -0.25, 1e-3, 3.0], np.float32)
+    cfg = oracle.scaler_cfg(False)
+    st = oracle.state_init(cfg)
+    hp = oracle.hparams()
+    R = np.zeros(4, np.float32)
+    master, m, v = p0.copy(), np.zeros(4, np.float32), np.zeros(4, np.float32)
+    params = np.zeros(4, np.uint16)
+    z = np.zeros(4, np.uint16)
+    for _ in range(50):
+        sc = oracle.step([z, z], BF16, 1 << 40, R, master, m, v, params, BF16, cfg, hp, st)
+    assert not m.any() and not v.any()
+    ref = p0.astype(np.float64) * (1 - 6e-5 * 0.01) ** 50
+    # fp32 arithmetic: the decay factor 1 - 6e-7 is held in fp32 (within 2^-25 of the
+    # exact value) and each of the 50 products rounds by at most 2^-24 relative, so
+    # |err| <= 50 * (2^-25 + 2^-24) ~ 4.5e-6; dropping the decay would be off by 3e-5.
+    np.testing.assert_allclose(master, ref, rtol=50 * (2.0 ** -25 + 2.0 ** -24))
+    assert np.all(np.abs(master - p0) > 2.5e-5 * np.abs(p0))
+    assert sc.adam_t == 50
+
+
+def test_matches_torch_cpu_adamw_with_clipping():
+    # W = 1 and no loss scaling: the step is torch's clip_grad_norm_ followed by
+    # torch.optim.AdamW. Torch runs in fp64 here (its fp32 norm alone is off by ~1e-6),
+    # so it stands for the exact result; the fp32 oracle must stay within 1e-6 of it.
+    rng = np.random.default_rng(7)
+    n = 1 << 16
+    p0 = rng.normal(0, 0.02, n).astype(np.float32)
+    tp = torch.nn.Parameter(torch.from_numpy(p0.astype(np.float64)))
+    opt = torch.optim.AdamW([tp], lr=6e-5, betas=(0.9, 0.999), eps=1e-8, weight_decay=0.01)
+    cfg = oracle.scaler_cfg(False)
+    hp = oracle.hparams()
+    st = oracle.state_init(cfg)
+    R = np.zeros(n, np.float32)
+    master, m, v = p0.copy(), np.zeros(n, np.float32), np.zeros(n, np.float32)
+    params = np.zeros(n, np.uint16)
+    clipped = 0
+    for t in range(1, 7):
+        sigma = 1e-2 if t % 2 else 1e-3  # norm ~2.6 (clipped) and ~0.26 (not clipped)
+        gh = oracle.f32_to_half(rng.normal(0, sigma, n).astype(np.float32), BF16)
+        sc = oracle.step([gh], BF16, 1 << 40, R, master, m, v, params, BF16, cfg, hp, st)
+        tp.grad = torch.from_numpy(oracle.half_to_f32(gh, BF16).astype(np.float64))
+        tn = torch.nn.utils.clip_grad_norm_([tp], 1.0)
+        assert abs(float(tn) - sc.norm) / sc.norm < 1e-12
+        clipped += sc.clip_coef < 1.0
+        opt.step()
+        s = opt.state[tp]
+        for mine, theirs in ((master, tp.detach()), (m, s["exp_avg"]), (v, s["exp_avg_sq"])):
+            theirs = theirs.numpy()
+            floor = np.sqrt(np.mean(theirs ** 2))
+            err = np.abs(mine - theirs) / np.maximum(np.abs(theirs), floor)
+            assert err.max() <= 1e-6, (t, err.max())
+    assert clipped == 3
+
+
+# ----------------------------------------------------------------------------- loss scaler
+
+def _expand(groups, cast):
+    out = []
+    for g in groups.split():
+        v, k = g.split("x")
+        out += [cast(v)] * int(k)
+    return out
+
+
+def _traces():
+    rows = []
+    with open(os.path.join(GOLDEN, "scaler_traces.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            name, cfgs, flags, scales, final, hyst, adam = [x.strip() for x in line.split("|")]
+            dyn, p, w, h, mn = cfgs.split()
+            rows.append(dict(name=name, dynamic=int(dyn), power=int(p), window=int(w),
+                             hyst=int(h), min_scale=float(mn),
+                             flags=_expand(flags, int), scales=_expand(scales, float),
+                             final=float(final), final_hyst=int(hyst), adam=int(adam)))
+    return rows
+
+
+@pytest.mark.parametrize("tr", _traces(), ids=lambda t: t["name"])
+def test_scaler_golden_traces(tr):
+    cfg = oracle.scaler_cfg(bool(tr["dynamic"]), tr["power"], tr["window"], tr["hyst"],
+                            tr["min_scale"])
+    hp = oracle.hparams()
+    st = oracle.state_init(cfg)
+    used = []
+    for f in tr["flags"]:
+        sc = oracle.finalize(math.inf if f else 1.0, bool(f), cfg, hp, st)
+        used.append(sc.scale_used)
+        assert sc.skipped == f
+    assert used == tr["scales"]
+    assert st.scale == tr["final"] and st.cur_hysteresis == tr["final_hyst"]
+    assert st.adam_t == tr["adam"] and st.iter == len(tr["flags"])
+
+
+def test_scaler_invariants_all_short_sequences():
+    cfg = oracle.scaler_cfg(True, 16, 3, 2, 1.0)
+    hp = oracle.hparams()
+    for L in range(1, 13):
+        for code in range(1 << L):
+            st = oracle.state_init(cfg)
+            prev = st.scale
+            halvings = 0
+            for i in range(L):
+                f = (code >> i) & 1
+                sc = oracle.finalize(math.inf if f else 1.0, bool(f), cfg, hp, st)
+                assert sc.scale_used == prev
+                nxt = st.scale
+                assert nxt >= 1.0 and math.frexp(nxt)[0] == 0.5  # a power of two
+                if f:
+                    assert nxt in (prev, max(prev / 2, 1.0))
+                    halvings += nxt < prev
+                else:
+                    assert nxt in (prev, prev * 2)
+                prev = nxt
+            assert st.adam_t == L - bin(code).count("1")
+            assert halvings <= bin(code).count("1")
+
+
+# ----------------------------------------------------------------------------- planner
+
+def _brute_plan(numels, W, B, A):
+    N = sum(numels)
+    n_pad = N
+    while n_pad % (W * A):
+        n_pad += 1
+    P = n_pad // W
+    owner = [i // P for i in range(n_pad)]
+    bucket = [i // B for i in range(n_pad)]
+    return N, n_pad, P, owner, bucket
+
+
+@pytest.mark.parametrize("seed", range(25))
+def test_planner_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    nt = int(rng.integers(0, 6))
+    numels = [int(x) for x in rng.integers(0, 60, nt)]
+    W = int(rng.choice([1, 2, 3, 4, 8, 16]))
+    A = int(rng.choice([1, 2, 8]))
+    B = int(rng.integers(1, 80))
+    pl = oracle.plan(numels, W, B, A)
+    N, n_pad, P, owner, bucket = _brute_plan(numels, W, B, A)
+    assert (pl.n, pl.n_pad, pl.p) == (N, n_pad, P)
+    assert pl.n_buckets == (max(bucket) + 1 if n_pad else 0)
+    segs = oracle.work_segments(pl.n_pad, W, B)
+    cover = np.zeros(n_pad, int)
+    for b, r, s, ln in segs:
+        for i in range(s, s + ln):
+            cover[i] += 1
+            assert owner[i] == r and bucket[i] == b
+    assert np.all(cover == 1)
+    flat_tensor = []
+    for t, n in enumerate(numels):
+        flat_tensor += [(t, k) for k in range(n)]
+    flat_tensor += [(-1, k) for k in range(n_pad - N)]
+    for r in range(W):
+        for t, off, flat, ln in oracle.partition(numels, n_pad, W, r):
+            for k in range(ln):
+                assert flat_tensor[flat + k] == (t, off + k)
+                assert owner[flat + k] == r
+
+
+def test_planner_config_sizes():
+    for name, nb in (("tiny", 1), ("enc", 1), ("gpt2", 2), ("llama7b", 14)):
+        wl = synthgen.workload(name)
+        pl = oracle.plan(wl.numels, wl.world, wl.bucket, wl.align)
+        assert pl.n == pl.n_pad == wl.n  # the graded tensor lists need no padding
+        assert pl.n_buckets == nb and pl.p * wl.world == pl.n_pad
+    with pytest.raises(ValueError):
+        oracle.plan([1, -1], 2, 10)
+    with pytest.raises(ValueError):
+        oracle.plan([1 << 62, 1 << 62], 2, 10)
+
+
+# ----------------------------------------------------------------------------- memory
+
+def _golden_memory():
+    d = {}
+    with open(os.path.join(GOLDEN, "memory_pages.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                k, v = line.split()
+                d[k] = float(v)
+    return d
+
+
+def test_memory_accounting_matches_pages():
+    g = _golden_memory()
+    psi = 7e9
+    ddp = oracle.memory_per_rank(psi, 8, 0)
+    z1 = oracle.memory_per_rank(psi, 8, 1)
+    assert 1 - z1["optimizer_state"] / ddp["optimizer_state"] == g["optimizer_state_saving_w8"]
+    big = 1 << 30
+    ddp_total = oracle.memory_per_rank(psi, big, 0)["total"]
+    assert abs(ddp_total / oracle.memory_per_rank(psi, big, 1)["total"] - g["zero1_ratio_limit"]) < 1e-6
+    assert abs(ddp_total / oracle.memory_per_rank(psi, big, 2)["total"] - g["zero2_ratio_limit"]) < 1e-6
+    # ZeRO-3 divides everything by W: a 320 GB footprint on 4 ranks is 80 GB each
+    psi320 = 320e9 / 16
+    assert oracle.memory_per_rank(psi320, 4, 3)["total"] / 1e9 == g["zero3_320gb_on_4"]
+    # four copies of ~268 MB of fp32 per layer exceed 1 GB (16 bytes per parameter)
+    psi_layer = g["encoder_layer_fp32_mb"] * 1e6 / 4
+    assert oracle.memory_per_rank(psi_layer, 1, 0)["total"] > 1e9
+    # stages only ever reduce per-rank memory
+    for W in (1, 2, 8, 64):
+        tot = [oracle.memory_per_rank(psi, W, s)["total"] for s in range(4)]
+        assert tot == sorted(tot, reverse=True)
