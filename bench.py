@@ -1,0 +1,499 @@
+#!/usr/bin/env python
+"""Benchmark of the ZeRO partitioned optimizer step on B200.
+
+One step = the whole hot path on one batch of synthetic gradients: reduce-scatter of
+every bucket of W replica gradients (fp32 rank-ordered sum + fp64 sum of squares),
+the finalize kernel (overflow, norm, clip, loss scaler, step constants) and the fused
+AdamW + half-cast update of every rank's partition (which is also the all-gather).
+
+Default workload: the Llama-7B-shaped tensor list (6,738,415,616 params, 291 tensors),
+W = 8 simulated ranks, bf16 gradients, reduce_bucket_size 5e8 (14 buckets). Replica
+buffers hold one bucket (2 slots of W x 5e8 bf16, generated before timing); fp32
+master / m / v / reduced gradient and the bf16 gathered buffer are resident
+(about 137 GB). Each step moves about 337 GB, far more than L2, so no flush is needed.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs an independent replica of the workload on its
+own GPU (the single-GPU step has no cross-GPU exchange); the time is the max over
+ranks and `value` counts the parameters all ranks updated.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ZeRO step params/s and achieved HBM GB/s vs ~8 TB/s peak, W=8 simulated ranks"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama7b",
+                    help="llama7b | gpt2 | enc | tiny | sweep")
+    ap.add_argument("--log2n", type=int, default=26, help="sweep: log2 of the parameter count")
+    ap.add_argument("--world", type=int, default=8, help="sweep: simulated ranks W")
+    ap.add_argument("--dtype", default="bf16", help="sweep: bf16 | fp16")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def get_workload(args):
+    import synthgen
+    if args.workload == "sweep":
+        return synthgen.sweep(args.log2n, args.world, args.dtype)
+    wl = synthgen.workload(args.workload)
+    return wl
+
+
+def schedule_bytes_per_param(W: int) -> int:
+    # reduce-scatter: W half reads + fp32 write; update: fp32 R, p, m, v reads, p, m, v
+    # writes and the half write
+    return 2 * W + 4 + 16 + 14
+
+
+def model_bytes_per_param(W: int) -> int:
+    return 2 * W + 26
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    with open(os.path.join(ROOT, "zero_sharded_mixed_replica_b200", "csrc", "kernels.cu"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    src_hash, traffic = None, None
+    with open(path) as f:
+        for line in f:
+            if line.startswith("kernels.cu sha256[:16]:"):
+                src_hash = line.split(":", 1)[1].strip()
+            if line.startswith("dram bytes per launch:"):
+                traffic = float(line.split(":", 1)[1].strip().split()[0])
+    if src_hash != kernel_source_hash():
+        return None
+    return traffic
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 100):
+        self.gpu_index = gpu_index
+        self.period_ms = period_ms
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 f"-lms", str(self.period_ms), "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.reader.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank: int, world_size: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    from synthgen import device as sdev
+    import zero_sharded_mixed_replica_b200 as zb
+
+    wl = get_workload(args)
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    s = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(s)
+    sh = s.cuda_stream
+    half = {"bf16": torch.bfloat16, "fp16": torch.float16}[wl.gdtype]
+
+    scaler = zb.scaler_cfg(wl.dynamic, wl.init_scale_power, wl.loss_scale_window,
+                           wl.hysteresis, wl.min_loss_scale)
+    adamw = zb.adamw_cfg(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.max_grad_norm)
+    opt = zb.ZeroOptimizer([t.shape for t in wl.tensors], wl.world, wl.bucket, wl.gdtype,
+                           wl.align, scaler, adamw, device=str(dev), stream=s)
+    plan = opt.plan
+    n_pad, W, nb = plan.n_pad, wl.world, plan.n_buckets
+    sdev.init_master(wl, opt.master, sh)
+    opt.cast_params()
+    # replica gradients: two slots of W bucket-sized buffers (or whole-model buffers
+    # when the model fits in one bucket)
+    L = min(wl.bucket, n_pad)
+    slots = [[torch.zeros(L, dtype=half, device=dev) for _ in range(W)] for _ in range(2)]
+    scale = float(2.0 ** wl.init_scale_power) if wl.dynamic else 1.0
+    for k in range(2):
+        sdev.fill_grads(wl, slots[k], 0, min(L, wl.n), k + 1, scale, sh)
+    torch.cuda.synchronize(dev)
+
+    ev_k1 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps * nb)]
+    ev_k3 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    ev_k2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+
+    def one_step(t: int, timed: int = -1):
+        bufs = slots[(t - 1) % 2] if wl.streaming else slots[0]
+        for b in range(nb):
+            if timed >= 0:
+                ev_k1[timed * nb + b][0].record(s)
+            opt.reduce_scatter_bucket(b, bufs, base_offset=b * wl.bucket if wl.streaming else 0)
+            if timed >= 0:
+                ev_k1[timed * nb + b][1].record(s)
+        if timed >= 0:
+            ev_k2[timed][0].record(s)
+        opt.step_finalize()
+        if timed >= 0:
+            ev_k2[timed][1].record(s)
+            ev_k3[timed][0].record(s)
+        opt.step_update()
+        if timed >= 0:
+            ev_k3[timed][1].record(s)
+
+    step_no = 0
+    for _ in range(args.warmup):
+        step_no += 1
+        one_step(step_no)
+    torch.cuda.synchronize(dev)
+    if world_size > 1:
+        dist.barrier()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    if world_size > 1:
+        dist.barrier()
+    t_wall0 = time.perf_counter()
+    start.record(s)
+    for i in range(args.steps):
+        step_no += 1
+        one_step(step_no, timed=i)
+    end.record(s)
+    torch.cuda.synchronize(dev)
+    t_wall = time.perf_counter() - t_wall0
+    if world_size > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms_total = start.elapsed_time(end)
+    res = opt.result()
+
+    k1_ms = [a.elapsed_time(b) for a, b in ev_k1]
+    k2_ms = [a.elapsed_time(b) for a, b in ev_k2]
+    k3_ms = [a.elapsed_time(b) for a, b in ev_k3]
+
+    ms_max = ms_total
+    if world_size > 1:
+        tt = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_max = float(tt.item())
+
+    out = None
+    if rank == 0:
+        ms_step = ms_max / args.steps
+        params_step = plan.n  # parameters updated per step (padding excluded)
+        value = params_step * args.steps * world_size / (ms_max / 1e3)
+        peak, peak_kind = measured_peaks()
+        k3_avg = sum(k3_ms) / len(k3_ms)
+        k3_bytes = 30 * n_pad  # R, p, m, v read (16 B) + p, m, v write (12 B) + half (2 B)
+        k3_gbs = k3_bytes / (k3_avg / 1e3) / 1e9
+        full_b = [k1_ms[i] for i in range(len(k1_ms)) if plan.bucket(i % nb)[1] == wl.bucket] or k1_ms
+        k1_avg = sum(full_b) / len(full_b)
+        k1_bytes = (2 * W + 4) * plan.bucket(0)[1]
+        sched_gbs = schedule_bytes_per_param(W) * n_pad / (ms_step / 1e3) / 1e9
+        model_gbs = model_bytes_per_param(W) * plan.n / (ms_step / 1e3) / 1e9
+        traffic = profiled_traffic("adamw_cast", wl.name)
+        out = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "params/s",
+            "n_gpus": world_size,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16+fp32" if wl.gdtype == "bf16" else "fp16+fp32",
+            "data": "synthetic (seeded Philox gradients and init; random-init weights of the shape list)",
+            "config": {
+                "workload": f"{wl.name}_w{W}",
+                "params": plan.n,
+                "tensors": len(wl.tensors),
+                "W": W,
+                "reduce_bucket_size": wl.bucket,
+                "buckets": nb,
+                "grad_dtype": wl.gdtype,
+                "replica_buffers": "bucket-sized, 2 slots" if wl.streaming else "resident",
+                "l2": f"no flush: each step moves {schedule_bytes_per_param(W) * n_pad / 1e9:.0f} GB, inputs >> 126 MB L2",
+                "parallelism": f"replicas x{world_size} (simulated dp{W} per GPU)",
+            },
+            "hbm_gbs_schedule": sched_gbs,
+            "hbm_gbs_model": model_gbs,
+            "frac_of_8tbs_schedule": sched_gbs / 8000.0,
+            "frac_of_peak_schedule": sched_gbs / peak,
+            "stage_ms": {"reduce_scatter_total": sum(k1_ms) / args.steps,
+                         "finalize": sum(k2_ms) / len(k2_ms),
+                         "adamw_cast": k3_avg},
+            "reduce_scatter_gbs": k1_bytes / (k1_avg / 1e3) / 1e9,
+            "roofline": {
+                "kernel": "adamw_cast_kernel",
+                "bound": "hbm",
+                "achieved": k3_gbs,
+                "peak": peak,
+                "peak_kind": peak_kind,
+                "unit": "GB/s",
+                "frac": k3_gbs / peak,
+                "traffic": traffic,
+                "algorithmic_bytes_per_launch": k3_bytes,
+            },
+            "gpu_launches": args.steps * (nb + 2),
+            "clocks": clocks,
+            "wall_s_timed": t_wall,
+            "last_result": {k: res[k] for k in ("global_norm", "clip_coef", "adam_t", "skipped")},
+        }
+    del opt, slots
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_e2e(args, wl, local_rank: int):
+    """Same metric through the public C ABI with HOST gradient buffers: every bucket's
+    replica slices are copied host -> device (pinned) inside the timed region by
+    zero_reduce_scatter_bucket_host, and the step result is read back each step."""
+    import numpy as np
+    import torch
+
+    import synthgen
+    from synthgen import device as sdev
+    import zero_sharded_mixed_replica_b200 as zb
+
+    dev = torch.device("cuda", local_rank)
+    s = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(s)
+    scaler = zb.scaler_cfg(wl.dynamic, wl.init_scale_power, wl.loss_scale_window,
+                           wl.hysteresis, wl.min_loss_scale)
+    adamw = zb.adamw_cfg(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.max_grad_norm)
+    opt = zb.ZeroOptimizer([t.shape for t in wl.tensors], wl.world, wl.bucket, wl.gdtype,
+                           wl.align, scaler, adamw, device=str(dev), stream=s)
+    plan = opt.plan
+    W, nb = wl.world, plan.n_buckets
+    sdev.init_master(wl, opt.master, s.cuda_stream)
+    opt.cast_params()
+    L = min(wl.bucket, plan.n_pad)
+    half = {"bf16": torch.bfloat16, "fp16": torch.float16}[wl.gdtype]
+    # pinned host gradients: the same two-slot recipe as the device-resident run
+    host = [[torch.empty(L, dtype=torch.int16).pin_memory() for _ in range(W)] for _ in range(2)]
+    for k in range(2):
+        for r in range(W):
+            synthgen.grads_host(0, min(L, wl.n), wl.seed, r, wl.slot(k + 1), wl.grad_sigma,
+                                wl.spike_frac, 1.0, wl.dtype_code,
+                                out=host[k][r].numpy().view(np.uint16))
+    staging = [torch.empty(L, dtype=half, device=dev) for _ in range(W)]
+    h2d = 0
+
+    def one(t):
+        nonlocal h2d
+        hb = host[(t - 1) % 2]
+        ptrs = [h.data_ptr() for h in hb]
+        for b in range(nb):
+            opt.reduce_scatter_bucket_host(b, ptrs, b * wl.bucket if wl.streaming else 0, staging)
+            h2d += W * plan.bucket(b)[1] * 2
+        opt.step()
+        return opt.result()  # device -> host read of the step result (synchronises)
+
+    one(1)
+    torch.cuda.synchronize(dev)
+    h2d = 0
+    t0 = time.perf_counter()
+    for i in range(args.e2e_steps):
+        one(i + 2)
+    dt = time.perf_counter() - t0
+    out = {"value": plan.n * args.e2e_steps / dt, "unit": "params/s",
+           "h2d_bytes_per_step": h2d // args.e2e_steps,
+           "d2h_bytes_per_step": ctypes.sizeof(zb.StepResult),
+           "steps": args.e2e_steps,
+           "path": "zero_reduce_scatter_bucket_host (pinned host replicas) + zero_step + zero_get_result"}
+    del opt, staging, host
+    torch.cuda.empty_cache()
+    return out
+
+
+# ---------------------------------------------------------------------------- oracle arm
+
+def oracle_sample_run(wl, seconds: float, max_steps: int = 0, warmup: int = 0):
+    """The CPU oracle, as it stands (single-threaded C), on a bounded sample of the
+    workload: the first `n` elements of the first bucket, all W replicas, one step of
+    reduce + sum of squares + finalize + AdamW/cast per iteration. Inputs are drawn
+    before timing. Returns (params/s, sample description, steps, seconds)."""
+    import numpy as np
+
+    import oracle
+    import synthgen
+
+    n = min(1 << 24, wl.n)
+    dt = wl.dtype_code
+    grads = [synthgen.grads_host(0, n, wl.seed, r, wl.slot(1), wl.grad_sigma, wl.spike_frac,
+                                 1.0, dt) for r in range(wl.world)]
+    master = synthgen.master_random_host(0, n, wl.seed, wl.init_sigma)
+    m = np.zeros(n, np.float32)
+    v = np.zeros(n, np.float32)
+    R = np.zeros(n, np.float32)
+    params = oracle.f32_to_half(master, dt)
+    cfg, hp = oracle.workload_cfg(wl)
+    st = oracle.state_init(cfg)
+    for _ in range(warmup):
+        oracle.step(grads, dt, wl.bucket, R, master, m, v, params, dt, cfg, hp, st)
+    steps = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.step(grads, dt, wl.bucket, R, master, m, v, params, dt, cfg, hp, st)
+        steps += 1
+        el = time.perf_counter() - t0
+        if (max_steps and steps >= max_steps) or (not max_steps and el >= seconds):
+            break
+    desc = (f"{n} params ({wl.name} flat indices 0..{n - 1}), W={wl.world} {wl.gdtype} replicas, "
+            f"{steps} full oracle steps (reduce, sum of squares, finalize, AdamW + cast)")
+    return n * steps / el, desc, steps, el
+
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return None
+    wl = get_workload(args)
+    val, desc, steps, el = oracle_sample_run(wl, 0, max_steps=args.steps, warmup=args.warmup)
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": val,
+        "unit": "params/s",
+        "n_gpus": args.gpus,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": el / steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16+fp32" if wl.gdtype == "bf16" else "fp16+fp32",
+        "data": "synthetic (seeded Philox gradients and init)",
+        "config": {"workload": f"{wl.name}_w{wl.world}", "params": wl.n, "W": wl.world,
+                   "reduce_bucket_size": wl.bucket},
+        "cpu_baseline": {"value": val, "unit": "params/s", "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": val, "unit": "params/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world_size = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        out = run_reference(args, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world_size > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    out = run_ours(args, rank, world_size, local_rank)
+    if rank == 0:
+        wl = get_workload(args)
+        if not args.no_e2e and world_size == 1:
+            out["e2e"] = run_e2e(args, wl, local_rank)
+        elif not args.no_e2e:
+            out["e2e"] = None
+        if not args.no_cpu_baseline and world_size == 1:
+            val, desc, steps, el = oracle_sample_run(wl, args.cpu_seconds)
+            out["cpu_baseline"] = {"value": val, "unit": "params/s", "cores": 1, "kind": "oracle",
+                                   "sample": desc, "host_cpu_count": os.cpu_count()}
+        print(json.dumps(out), flush=True)
+    if world_size > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,264 @@
+/*
+ * zero_b200.h -- C ABI of libzero_b200.so: the ZeRO partitioned mixed-precision
+ * optimizer step on one B200 (sm_100a), with W data-parallel ranks simulated as W
+ * replica gradient buffers and W owned partitions in the same GPU's memory.
+ *
+ * One step, in order:
+ *   1. zero_reduce_scatter_bucket(b) for every bucket b: sum the W replica gradients
+ *      of the bucket in fp32 in rank order; each rank's slice of the result is its
+ *      reduced gradient partition. Also accumulates the fp64 sum of squares.
+ *   2.-4. zero_step: overflow (inf/NaN) detection, dynamic loss-scale update, global
+ *      L2-norm clipping, and AdamW on every rank's fp32 master / m / v partition,
+ *      writing the rounded half-precision parameters straight into the gathered
+ *      buffer (the all-gather of step 5 costs nothing extra on one GPU).
+ *   5. zero_all_gather: optional copies of the gathered buffer into per-rank buffers.
+ *
+ * Sources (web pages; titles and sections):
+ *  [Z1] "ZeRO技术解析：大模型分布式训练的革命性突破" (ZeRO explained): 1.2.1-1.2.3 (the three
+ *       stages: optimizer state, gradients and parameters partitioned), 2.1 (parameters
+ *       split automatically into N parts, gradients reduce-scattered in backward, each
+ *       GPU updates only its own partition, bucketed communication), 2.2 (gradient
+ *       buckets via reduce_bucket_size; batched all-gather of large matrices), 3.1
+ *       (AdamW, lr 6e-5, weight_decay 0.01), 3.3 (fp16 loss_scale_window 100,
+ *       hysteresis 2), 5.1 (initial_scale_power 16, min_loss_scale 1), 5.2
+ *       (reduce_bucket_size 5e8, contiguous_gradients), 6 (gradient_clipping 1.0,
+ *       reduce_bucket_size 2e8).
+ *  [Z2] "大模型分片训练：ZeRO-3策略在PyTorch中的实现" (ZeRO-3 in PyTorch): memory arithmetic of
+ *       one encoder layer, the per-stage saving table, the ds_config with
+ *       allgather_bucket_size and reduce_scatter, deepspeed.initialize.
+ *  [Z3] "ZeRO 和分片优化器" (ZeRO and sharded optimizers): gradients are reduce-scattered
+ *       so each GPU keeps the slice for its own parameters; Adam keeps first and second
+ *       moments beside fp32 master weights (FAQ).
+ *
+ * Conventions for every call
+ *  - Return value: ZERO_OK (0) or a negative ZERO_E* code; zero_last_error() then gives
+ *    a message (thread-local, valid until the next call on the same thread). Nothing
+ *    throws across this boundary.
+ *  - Ownership: the caller allocates and owns every device buffer, the workspace and
+ *    the stream. The library owns only the plan (host memory). It never allocates
+ *    device memory and never synchronises, except zero_get_result.
+ *  - Streams: `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *    stream. All device work of a call is enqueued on that stream, in order.
+ *  - Device pointers must be 16-byte aligned (ZERO_EALIGN otherwise).
+ *  - Conditions found on the device (overflow, a skipped step) are results, not errors.
+ *  - Calls on one plan must not run concurrently from several host threads.
+ */
+#ifndef ZERO_B200_H
+#define ZERO_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ZERO_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define ZERO_API __attribute__((visibility("default")))
+#else
+#define ZERO_API
+#endif
+
+/* error codes */
+#define ZERO_OK 0
+#define ZERO_EINVAL (-1) /* null pointer, W outside [1, ZERO_MAX_WORLD], negative dim, bucket out of range, bad hyperparameter */
+#define ZERO_EALIGN (-2) /* a device pointer or replica base offset breaks the alignment rule */
+#define ZERO_ERANGE (-3) /* the parameter count overflows int64 */
+#define ZERO_ESTATE (-4) /* call out of order: a bucket reduced twice, or a step before every bucket was reduced */
+#define ZERO_ECUDA (-5)  /* a CUDA launch or copy failed; the message names the CUDA error */
+#define ZERO_ENOMEM (-6) /* host allocation for the plan failed */
+
+/* element types of gradients and gathered parameters */
+#define ZERO_BF16 0
+#define ZERO_FP16 1
+
+#define ZERO_MAX_WORLD 16 /* simulated ranks per reduce-scatter launch */
+
+typedef struct zero_plan zero_plan; /* opaque; host memory owned by the library */
+
+typedef struct {
+  int64_t n;          /* parameters: sum of tensor numels in declared order        */
+  int64_t n_pad;      /* ceil(n / (W*align)) * W*align                              */
+  int64_t p;          /* partition length n_pad / W                                 */
+  int64_t n_buckets;  /* ceil(n_pad / bucket_size)                                  */
+  int64_t n_segments; /* work segments: bucket intersect partition                  */
+  int64_t n_tensors;
+  int64_t bucket_size; /* reduce_bucket_size in elements                            */
+  int32_t world_size;  /* W                                                         */
+  int32_t align;       /* alignment unit A in elements                              */
+} zero_plan_info;
+
+/* A piece of one tensor inside one rank's partition; tensor == -1 is zero padding. */
+typedef struct {
+  int64_t tensor;
+  int64_t offset_in_tensor;
+  int64_t flat_offset;
+  int64_t length;
+} zero_segment;
+
+/* bucket intersect partition */
+typedef struct {
+  int64_t bucket;
+  int64_t rank;
+  int64_t start; /* flat index */
+  int64_t length;
+} zero_work_segment;
+
+/* Loss scaler ([Z1] 3.3, 5.1). dynamic=0: a fixed scale `static_scale` (1 for bf16). */
+typedef struct {
+  int32_t dynamic;
+  int32_t initial_scale_power; /* scale starts at 2^initial_scale_power            */
+  int64_t loss_scale_window;   /* good steps between growths                        */
+  int32_t hysteresis;          /* overflows tolerated before backing off            */
+  float min_loss_scale;
+  float scale_factor;          /* growth / back-off factor, normally 2              */
+  float static_scale;
+} zero_scaler_cfg;
+
+/* AdamW ([Z1] 3.1) and clipping ([Z1] 6). max_grad_norm <= 0 disables clipping. */
+typedef struct {
+  double lr, beta1, beta2, eps, weight_decay, max_grad_norm;
+} zero_adamw_cfg;
+
+typedef struct {
+  double global_norm; /* L2 norm of the unscaled gradient before clipping           */
+  double sumsq;       /* fp64 sum of squares of the scaled reduced gradient         */
+  float clip_coef;    /* min(1, max_grad_norm / (global_norm + 1e-6))                */
+  float scale_used;   /* loss scale this step's gradients carried                    */
+  float next_scale;   /* loss scale after the scaler transition                      */
+  float k;            /* fp32 multiplier applied to the reduced gradient: clip/scale */
+  int32_t overflow;   /* a reduced gradient was inf or NaN                           */
+  int32_t skipped;    /* the update was skipped (overflow)                           */
+  int32_t hysteresis; /* hysteresis budget after the step                            */
+  int32_t reserved;
+  int64_t iter;       /* scaler iterations so far (every step)                       */
+  int64_t adam_t;     /* applied AdamW steps so far                                  */
+} zero_step_result;
+
+/* bytes per rank */
+typedef struct {
+  double params, grads, optimizer_state, total;
+} zero_memory;
+
+/* ---------------------------------------------------------------- planning (host only)
+ * zero_plan_create: [Z1] 2.1 (parameters split automatically into N = W parts, one per
+ * GPU; communication in buckets), [Z1] 4.1 table (ZeRO partitions by dynamic bucket,
+ * not by module), [Z1] 2.2 / 5.2 / 6 (reduce_bucket_size).
+ * Tensors are flattened in the order given (tensor t has ndims[t] dims read in turn
+ * from `dims`; ndims 0 means a scalar), padded with zeros to n_pad, a multiple of
+ * W*align_elems; rank r owns the flat range [r*p, (r+1)*p); bucket b is
+ * [b*B, min((b+1)*B, n_pad)) with B = reduce_bucket_size ELEMENTS.
+ * Errors: EINVAL (null out, world_size outside [1, 16], bucket < 1, align < 1, a
+ * negative dim), ERANGE (n overflows), ENOMEM. n_tensors may be 0 (an empty plan). */
+ZERO_API int zero_plan_create(const int64_t* dims, const int32_t* ndims, int32_t n_tensors,
+                     int32_t world_size, int64_t reduce_bucket_size, int32_t align_elems,
+                     zero_plan** out);
+ZERO_API void zero_plan_destroy(zero_plan* plan);
+ZERO_API int zero_plan_get_info(const zero_plan* plan, zero_plan_info* out);
+/* flat offset and numel of tensor t */
+ZERO_API int zero_plan_tensor(const zero_plan* plan, int32_t t, int64_t* flat_offset, int64_t* numel);
+/* flat start and length of bucket b */
+ZERO_API int zero_plan_bucket(const zero_plan* plan, int64_t b, int64_t* start, int64_t* length);
+/* Work segments (bucket-major, then rank). Writes min(cap, total) rows; *count = total. */
+ZERO_API int zero_plan_work_segments(const zero_plan* plan, zero_work_segment* out, int64_t cap,
+                            int64_t* count);
+/* Partition table of one rank ([Z3]: each GPU owns one slice). Same cap/count rule. */
+ZERO_API int zero_plan_partition(const zero_plan* plan, int32_t rank, zero_segment* out, int64_t cap,
+                        int64_t* count);
+/* Model-state bytes per rank for ZeRO stage 0..3 on this plan's W ranks, with half
+ * params and grads and fp32 master + m + v ([Z2] memory arithmetic and stage table,
+ * [Z1] 1.2.1: 8-way optimizer-state partitioning saves 87.5%). Partitioned items take
+ * p elements per rank, replicated ones n_pad. */
+ZERO_API int zero_plan_memory(const zero_plan* plan, int32_t stage, zero_memory* out);
+
+/* ---------------------------------------------------------------- device state
+ * Device workspace: scaler state, step constants, per-block partial sums of squares
+ * and the step result. The caller allocates zero_workspace_bytes() of device memory
+ * (16-byte aligned) and keeps it for the life of the optimizer. */
+ZERO_API int zero_workspace_bytes(const zero_plan* plan, size_t* bytes);
+/* Writes the initial scaler state and zero step counters into the workspace
+ * ([Z1] 3.3, 5.1): scale 2^initial_scale_power (dynamic) or static_scale, hysteresis
+ * budget full. Also resets the plan's per-step bookkeeping. EINVAL on a bad config. */
+ZERO_API int zero_state_init(zero_plan* plan, void* workspace, const zero_scaler_cfg* cfg,
+                    void* stream);
+/* Writes the half-precision copy of `master` (n_pad fp32) into the gathered buffer
+ * `params` (n_pad half): round to nearest even. Used once after initialisation or a
+ * load; steps keep the buffer current themselves. */
+ZERO_API int zero_cast_params(const zero_plan* plan, const float* master, void* params,
+                     int32_t param_dtype, void* stream);
+
+/* ---------------------------------------------------------------- the step
+ * zero_reduce_scatter_bucket ([Z1] 2.1 gradients reduce-scattered in backward; [Z1] 2.2
+ * reduce_bucket_size; [Z3] each GPU keeps the summed slice for its own parameters):
+ *   reduced[i] = ((g_0[i] + g_1[i]) + ...) + g_{W-1}[i]   for i in bucket b,
+ * each half converted exactly to fp32 and the sum taken in fp32 in rank order, written
+ * at the same flat index of `reduced` (n_pad fp32; rank r's slice [r*p, (r+1)*p) is its
+ * reduced gradient partition). The fp64 sum of squares of those values goes to the
+ * workspace (it yields both the global norm and the overflow flag).
+ *   replica_grads: HOST array of W device pointers; replica_grads[r][j] holds flat index
+ *   replica_base_offset + j, so a caller may pass bucket-sized buffers with
+ *   replica_base_offset = bucket start, or whole-model buffers with 0. Every replica
+ *   pointer and `reduced` must be 16-byte aligned. replica_base_offset must be <= the
+ *   bucket start.
+ * Each bucket must be reduced exactly once per step (ESTATE on a repeat). */
+ZERO_API int zero_reduce_scatter_bucket(zero_plan* plan, int64_t bucket, int32_t grad_dtype,
+                               const void* const* replica_grads, int64_t replica_base_offset,
+                               float* reduced, void* workspace, void* stream);
+
+/* Same as zero_reduce_scatter_bucket, but the replica gradients are in pinned HOST
+ * memory: each replica's bucket slice is first copied (cudaMemcpyAsync, host to device,
+ * on `stream`) into device_staging[r] (bucket-sized device buffers, W of them), then
+ * reduced. host_replica_grads[r][j] holds flat index host_base_offset + j. */
+ZERO_API int zero_reduce_scatter_bucket_host(zero_plan* plan, int64_t bucket, int32_t grad_dtype,
+                                    const void* const* host_replica_grads,
+                                    int64_t host_base_offset, void* const* device_staging,
+                                    float* reduced, void* workspace, void* stream);
+
+/* zero_step = zero_step_finalize + zero_step_update.
+ * zero_step_finalize (one CTA): S = sum of the partial sums in a fixed order; overflow
+ * = S not finite (any inf/NaN reduced gradient makes S inf or NaN); norm = sqrt(S)/scale
+ * in fp64; clip c = max_grad_norm/(norm + 1e-6) when below 1 ([Z1] 6); k = fp32(c/scale)
+ * folds unscale and clip into one multiply; loss-scaler transition ([Z1] 3.3, 5.1): on
+ * overflow, a hysteresis budget <= 1 divides the scale by the factor (not below
+ * min_loss_scale), otherwise the budget drops by one; on a good step the scale grows
+ * and the budget refills when (iter - last_overflow_iter) is a multiple of
+ * loss_scale_window. An overflowing step is skipped whole (master, m, v, params and
+ * adam_t unchanged); otherwise adam_t += 1 and the bias corrections 1 - beta^t are
+ * formed in fp64. ESTATE unless every bucket was reduced once since the last step.
+ * zero_step_update (AdamW on every owned partition, [Z1] 2.1 and 3.1, [Z3] FAQ), for
+ * every flat index i, in fp32 with each operation rounded (no fused multiply-add):
+ *   g = reduced[i]*k; m = b1*m + (1-b1)*g; v = b2*v + (1-b2)*(g*g);
+ *   p = p*(1 - lr*wd) - lr * ((m/bc1) / (sqrt(v/bc2) + eps));
+ *   params[i] = round_to_nearest_even_half(p)   (the fused all-gather write)
+ * It does nothing when the finalize step decided to skip. master, exp_avg, exp_avg_sq
+ * and reduced are n_pad fp32; params is the n_pad half gathered buffer. */
+ZERO_API int zero_step(zero_plan* plan, const zero_adamw_cfg* cfg, float* master, float* exp_avg,
+              float* exp_avg_sq, const float* reduced, void* params, int32_t param_dtype,
+              void* workspace, void* stream);
+ZERO_API int zero_step_finalize(zero_plan* plan, const zero_adamw_cfg* cfg, void* workspace,
+                       void* stream);
+ZERO_API int zero_step_update(zero_plan* plan, float* master, float* exp_avg, float* exp_avg_sq,
+                     const float* reduced, void* params, int32_t param_dtype,
+                     const void* workspace, void* stream);
+
+/* zero_all_gather ([Z1] 2.1 parameters gathered by allgather; [Z1] 2.2 batched
+ * all-gather; [Z2] allgather_bucket_size): after zero_step the gathered buffer `params`
+ * already holds every rank's partition, so n_dst = 0 is a no-op. With n_dst > 0 the
+ * full buffer is copied into each rank_params[d] (n_pad halves each, HOST array of
+ * device pointers), i.e. the per-rank replicas a multi-process run would hold. */
+ZERO_API int zero_all_gather(const zero_plan* plan, const void* params, void* const* rank_params,
+                    int32_t n_dst, int32_t param_dtype, void* stream);
+
+/* Copies the step result out of the workspace and synchronises `stream`. */
+ZERO_API int zero_get_result(const void* workspace, zero_step_result* out, void* stream);
+
+ZERO_API const char* zero_last_error(void);
+ZERO_API int zero_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZERO_B200_H */

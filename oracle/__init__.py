@@ -404,8 +404,14 @@ def streaming_scalars(wl, steps: Optional[int] = None, chunk: int = 1 << 24) -> 
     cfg, hp = workload_cfg(wl)
     st = state_init(cfg)
     res = []
+    cache = {}
     for t in range(1, (steps or wl.steps) + 1):
-        parts = streaming_slot_partials(wl, pl, t, step_grad_scale(wl, st), chunk)
+        # steps that draw the same slot at the same scale with no +inf sites see the
+        # same bucket contents: their partial sums are computed once
+        key = (wl.slot(t), step_grad_scale(wl, st)) if not wl.inf_sites.get(t) else ("t", t)
+        if key not in cache:
+            cache[key] = streaming_slot_partials(wl, pl, t, step_grad_scale(wl, st), chunk)
+        parts = cache[key]
         S, bad = 0.0, False
         for b in range(pl.n_buckets):
             Sb, badb = parts[_bucket_effective_len(pl, wl.n, b)]

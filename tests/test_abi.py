@@ -1,0 +1,143 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads and exports every
+symbol include/zero_b200.h declares, its planner agrees bit for bit with the oracle's
+independent planner, and misuse is rejected with the documented codes before any
+device work."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import synthgen
+import zero_sharded_mixed_replica_b200 as zb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    with open(os.path.join(ROOT, "include", "zero_b200.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"ZERO_API\s+[\w\s\*]*?\b(zero_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared_symbols()
+    assert len(names) >= 20
+    lib = ctypes.CDLL(zb.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert zb.zero_abi_version() == 1
+
+
+def _shapes_to_numels(shapes):
+    return [int(np.prod(s)) if len(s) else 1 for s in shapes]
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_planner_matches_oracle_planner(seed):
+    rng = np.random.default_rng(100 + seed)
+    shapes = []
+    for _ in range(int(rng.integers(0, 8))):
+        nd = int(rng.integers(0, 4))
+        shapes.append(tuple(int(x) for x in rng.integers(0, 9, nd)))
+    W = int(rng.integers(1, 17))
+    A = int(rng.choice([1, 2, 3, 8, 128]))
+    B = int(rng.integers(1, 3000))
+    plan = zb.Plan(shapes, W, B, A)
+    numels = _shapes_to_numels(shapes)
+    ref = oracle.plan(numels, W, B, A)
+    assert (plan.n, plan.n_pad, plan.p, plan.n_buckets) == (ref.n, ref.n_pad, ref.p, ref.n_buckets)
+    for t in range(len(shapes)):
+        assert plan.tensor(t) == (int(ref.offsets[t]), numels[t])
+    for b in range(plan.n_buckets):
+        s, ln = plan.bucket(b)
+        assert (s, ln) == ref.bucket_range(b)
+    segs = np.array(plan.work_segments(), dtype=np.int64).reshape(-1, 4)
+    assert np.array_equal(segs, oracle.work_segments(ref.n_pad, W, B))
+    for r in range(W):
+        got = np.array(plan.partition(r), dtype=np.int64).reshape(-1, 4)
+        assert np.array_equal(got, oracle.partition(numels, ref.n_pad, W, r)), r
+    assert plan.info.n_segments == len(segs)
+
+
+def test_config_plans():
+    for name in ("tiny", "enc", "gpt2", "llama7b"):
+        wl = synthgen.workload(name)
+        plan = zb.Plan([t.shape for t in wl.tensors], wl.world, wl.bucket, wl.align)
+        ref = oracle.plan(wl.numels, wl.world, wl.bucket, wl.align)
+        assert (plan.n, plan.n_pad, plan.p, plan.n_buckets) == (ref.n, ref.n_pad, ref.p, ref.n_buckets)
+        # memory per rank equals the oracle's accounting (no padding in these lists)
+        for stage in range(4):
+            got = plan.memory(stage)
+            want = oracle.memory_per_rank(float(wl.n), wl.world, stage)
+            for k in want:
+                assert got[k] == want[k]
+        assert plan.workspace_bytes() < 1 << 20
+
+
+def test_memory_saving_87_5_percent_at_w8():
+    plan = zb.Plan([(1 << 20,)], 8, 1 << 30)
+    ddp, z1 = plan.memory(0), plan.memory(1)
+    assert 1 - z1["optimizer_state"] / ddp["optimizer_state"] == 0.875
+
+
+def _code(fn, *a):
+    with pytest.raises(zb.ZeroError) as e:
+        fn(*a)
+    return e.value.code
+
+
+def test_plan_errors():
+    assert _code(zb.Plan, [(4,)], 0, 10) == zb.ZERO_EINVAL
+    assert _code(zb.Plan, [(4,)], 17, 10) == zb.ZERO_EINVAL
+    assert _code(zb.Plan, [(4,)], 2, 0) == zb.ZERO_EINVAL
+    assert _code(zb.Plan, [(4,)], 2, 10, 0) == zb.ZERO_EINVAL
+    assert _code(zb.Plan, [(4, -1)], 2, 10) == zb.ZERO_EINVAL
+    assert _code(zb.Plan, [(1 << 40, 1 << 40)], 2, 10) == zb.ZERO_ERANGE
+    assert _code(zb.Plan, [(1 << 62,), (1 << 62,)], 2, 10) == zb.ZERO_ERANGE
+    p = zb.Plan([(4,)], 2, 10)
+    assert _code(p.bucket, p.n_buckets) == zb.ZERO_EINVAL
+    assert _code(p.partition, 2) == zb.ZERO_EINVAL
+    assert _code(p.memory, 4) == zb.ZERO_EINVAL
+
+
+def test_empty_plan():
+    p = zb.Plan([], 4, 100)
+    assert (p.n, p.n_pad, p.n_buckets) == (0, 0, 0)
+    assert p.work_segments() == []
+    assert p.partition(0) == []
+    p = zb.Plan([(0, 5), ()], 2, 100, 1)  # an empty tensor and a scalar
+    assert (p.n, p.n_pad) == (1, 2)
+    assert p.partition(0) == [(1, 0, 0, 1)] and p.partition(1) == [(-1, 0, 1, 1)]
+
+
+def test_step_call_errors_before_any_device_work():
+    p = zb.Plan([(1024,)], 2, 512)
+    ws = 1 << 20  # fake, aligned device addresses: never dereferenced on these paths
+    R = 2 << 20
+    g = [3 << 20, 4 << 20]
+    assert _code(zb.zero_reduce_scatter_bucket, p, 2, "bf16", g, 0, R, ws) == zb.ZERO_EINVAL
+    assert _code(zb.zero_reduce_scatter_bucket, p, -1, "bf16", g, 0, R, ws) == zb.ZERO_EINVAL
+    assert _code(zb.zero_reduce_scatter_bucket, p, 0, 7, g, 0, R, ws) == zb.ZERO_EINVAL
+    assert _code(zb.zero_reduce_scatter_bucket, p, 0, "bf16", [g[0], 0], 0, R, ws) == zb.ZERO_EINVAL
+    assert _code(zb.zero_reduce_scatter_bucket, p, 0, "bf16", [g[0], g[1] + 2], 0, R, ws) == zb.ZERO_EALIGN
+    assert _code(zb.zero_reduce_scatter_bucket, p, 0, "bf16", g, 0, R + 4, ws) == zb.ZERO_EALIGN
+    assert _code(zb.zero_reduce_scatter_bucket, p, 0, "bf16", g, 0, None, ws) == zb.ZERO_EINVAL
+    assert _code(zb.zero_reduce_scatter_bucket, p, 1, "bf16", g, 600, R, ws) == zb.ZERO_EINVAL
+    cfg = zb.adamw_cfg()
+    # a step before every bucket was reduced
+    assert _code(zb.zero_step, p, cfg, R, R, R, R, R, "bf16", ws) == zb.ZERO_ESTATE
+    assert _code(zb.zero_step_update, p, R, R, R, R, R, "bf16", ws) == zb.ZERO_ESTATE
+    for bad in (zb.adamw_cfg(beta1=1.0), zb.adamw_cfg(eps=0.0), zb.adamw_cfg(lr=-1.0),
+                zb.adamw_cfg(beta2=float("nan")), zb.adamw_cfg(max_grad_norm=float("nan"))):
+        assert _code(zb.zero_step_finalize, p, bad, ws) == zb.ZERO_EINVAL
+    assert _code(zb.zero_step, p, cfg, R + 8, R, R, R, R, "bf16", ws) == zb.ZERO_EALIGN
+    assert _code(zb.zero_state_init, p, ws, zb.scaler_cfg(True, loss_scale_window=0)) == zb.ZERO_EINVAL
+    assert _code(zb.zero_state_init, p, ws, zb.scaler_cfg(True, hysteresis=0)) == zb.ZERO_EINVAL
+    assert _code(zb.zero_state_init, p, ws, zb.scaler_cfg(False, static_scale=0.0)) == zb.ZERO_EINVAL
+    assert _code(zb.zero_state_init, p, ws + 8, zb.scaler_cfg(False)) == zb.ZERO_EALIGN
+    assert _code(zb.zero_all_gather, p, R, [0], "bf16") == zb.ZERO_EINVAL
+    assert _code(zb.zero_all_gather, p, R, [R + 2], "bf16") == zb.ZERO_EALIGN
+    zb.zero_all_gather(p, R, [], "bf16")  # n_dst = 0: nothing to do

@@ -1,0 +1,324 @@
+"""Python binding of libzero_b200: the ZeRO partitioned mixed-precision optimizer step
+on B200 (sm_100a).
+
+This module only marshals arguments into the C ABI declared in ``include/zero_b200.h``;
+every step of the optimizer runs in the library's CUDA kernels. The functions carry
+the C names. There is no fallback: if ``libzero_b200.so`` is missing or fails to load,
+importing the binding raises.
+
+Device buffers are passed as integer device addresses (``tensor.data_ptr()``) or as
+torch tensors; streams as integer ``cudaStream_t`` handles (``stream.cuda_stream``)
+or torch streams; ``None`` means the legacy default stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Iterable, List, Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzero_b200.so")
+
+ZERO_OK = 0
+ZERO_EINVAL = -1
+ZERO_EALIGN = -2
+ZERO_ERANGE = -3
+ZERO_ESTATE = -4
+ZERO_ECUDA = -5
+ZERO_ENOMEM = -6
+ZERO_BF16 = 0
+ZERO_FP16 = 1
+ZERO_MAX_WORLD = 16
+DTYPES = {"bf16": ZERO_BF16, "fp16": ZERO_FP16}
+
+_ERR_NAMES = {ZERO_EINVAL: "EINVAL", ZERO_EALIGN: "EALIGN", ZERO_ERANGE: "ERANGE",
+              ZERO_ESTATE: "ESTATE", ZERO_ECUDA: "ECUDA", ZERO_ENOMEM: "ENOMEM"}
+
+
+class ZeroError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"{_ERR_NAMES.get(code, code)}: {message}")
+        self.code = code
+        self.message = message
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int64), ("n_pad", ctypes.c_int64), ("p", ctypes.c_int64),
+                ("n_buckets", ctypes.c_int64), ("n_segments", ctypes.c_int64),
+                ("n_tensors", ctypes.c_int64), ("bucket_size", ctypes.c_int64),
+                ("world_size", ctypes.c_int32), ("align", ctypes.c_int32)]
+
+
+class Segment(ctypes.Structure):
+    _fields_ = [("tensor", ctypes.c_int64), ("offset_in_tensor", ctypes.c_int64),
+                ("flat_offset", ctypes.c_int64), ("length", ctypes.c_int64)]
+
+
+class WorkSegment(ctypes.Structure):
+    _fields_ = [("bucket", ctypes.c_int64), ("rank", ctypes.c_int64),
+                ("start", ctypes.c_int64), ("length", ctypes.c_int64)]
+
+
+class ScalerCfg(ctypes.Structure):
+    _fields_ = [("dynamic", ctypes.c_int32), ("initial_scale_power", ctypes.c_int32),
+                ("loss_scale_window", ctypes.c_int64), ("hysteresis", ctypes.c_int32),
+                ("min_loss_scale", ctypes.c_float), ("scale_factor", ctypes.c_float),
+                ("static_scale", ctypes.c_float)]
+
+
+class AdamWCfg(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_double), ("beta1", ctypes.c_double),
+                ("beta2", ctypes.c_double), ("eps", ctypes.c_double),
+                ("weight_decay", ctypes.c_double), ("max_grad_norm", ctypes.c_double)]
+
+
+class StepResult(ctypes.Structure):
+    _fields_ = [("global_norm", ctypes.c_double), ("sumsq", ctypes.c_double),
+                ("clip_coef", ctypes.c_float), ("scale_used", ctypes.c_float),
+                ("next_scale", ctypes.c_float), ("k", ctypes.c_float),
+                ("overflow", ctypes.c_int32), ("skipped", ctypes.c_int32),
+                ("hysteresis", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("iter", ctypes.c_int64), ("adam_t", ctypes.c_int64)]
+
+    def as_dict(self) -> dict:
+        return {f: getattr(self, f) for f, _ in self._fields_ if f != "reserved"}
+
+
+class Memory(ctypes.Structure):
+    _fields_ = [("params", ctypes.c_double), ("grads", ctypes.c_double),
+                ("optimizer_state", ctypes.c_double), ("total", ctypes.c_double)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -c 'import __graft_entry__ as g; "
+            f"g.build()'` (nvcc, sm_100a). There is no CPU fallback.")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    P = ctypes.POINTER
+    sig = {
+        "zero_plan_create": [vp, vp, i32, i32, i64, i32, P(vp)],
+        "zero_plan_destroy": [vp],
+        "zero_plan_get_info": [vp, P(PlanInfo)],
+        "zero_plan_tensor": [vp, i32, P(i64), P(i64)],
+        "zero_plan_bucket": [vp, i64, P(i64), P(i64)],
+        "zero_plan_work_segments": [vp, vp, i64, P(i64)],
+        "zero_plan_partition": [vp, i32, vp, i64, P(i64)],
+        "zero_plan_memory": [vp, i32, P(Memory)],
+        "zero_workspace_bytes": [vp, P(ctypes.c_size_t)],
+        "zero_state_init": [vp, vp, P(ScalerCfg), vp],
+        "zero_cast_params": [vp, vp, vp, i32, vp],
+        "zero_reduce_scatter_bucket": [vp, i64, i32, vp, i64, vp, vp, vp],
+        "zero_reduce_scatter_bucket_host": [vp, i64, i32, vp, i64, vp, vp, vp, vp],
+        "zero_step": [vp, P(AdamWCfg), vp, vp, vp, vp, vp, i32, vp, vp],
+        "zero_step_finalize": [vp, P(AdamWCfg), vp, vp],
+        "zero_step_update": [vp, vp, vp, vp, vp, vp, i32, vp, vp],
+        "zero_all_gather": [vp, vp, vp, i32, i32, vp],
+        "zero_get_result": [vp, P(StepResult), vp],
+        "zero_last_error": [],
+        "zero_abi_version": [],
+    }
+    for name, args in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    L.zero_plan_destroy.restype = None
+    L.zero_last_error.restype = ctypes.c_char_p
+    return L
+
+
+lib = _load()
+
+
+def _check(rc: int) -> None:
+    if rc != ZERO_OK:
+        raise ZeroError(rc, (lib.zero_last_error() or b"").decode())
+
+
+def _addr(x) -> Optional[int]:
+    """Device address of an int, a torch tensor, or None."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s) -> Optional[int]:
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _ptr_array(ptrs: Sequence) -> ctypes.Array:
+    return (ctypes.c_void_p * len(ptrs))(*[_addr(p) for p in ptrs])
+
+
+def _dtype(dt) -> int:
+    return DTYPES[dt] if isinstance(dt, str) else int(dt)
+
+
+# ---------------------------------------------------------------------------- planning
+
+class Plan:
+    """Owns a zero_plan handle (host memory)."""
+
+    def __init__(self, shapes: Iterable[Sequence[int]], world_size: int,
+                 reduce_bucket_size: int, align: int = 128):
+        shapes = [tuple(int(d) for d in s) for s in shapes]
+        dims = [d for s in shapes for d in s]
+        ndims = [len(s) for s in shapes]
+        dims_arr = (ctypes.c_int64 * max(len(dims), 1))(*dims)
+        ndims_arr = (ctypes.c_int32 * max(len(ndims), 1))(*ndims)
+        h = ctypes.c_void_p()
+        _check(lib.zero_plan_create(dims_arr, ndims_arr, len(shapes), int(world_size),
+                                    int(reduce_bucket_size), int(align), ctypes.byref(h)))
+        self._h = h
+        self._destroy = lib.zero_plan_destroy  # kept for interpreter shutdown
+        self.shapes = shapes
+        inf = PlanInfo()
+        _check(lib.zero_plan_get_info(self._h, ctypes.byref(inf)))
+        self.info = inf
+
+    @property
+    def handle(self):
+        return self._h
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        destroy = getattr(self, "_destroy", None)
+        if h is not None and h.value and destroy is not None:
+            destroy(h)
+            self._h = None
+
+    # convenience views of the info
+    n = property(lambda self: self.info.n)
+    n_pad = property(lambda self: self.info.n_pad)
+    p = property(lambda self: self.info.p)
+    n_buckets = property(lambda self: self.info.n_buckets)
+    world_size = property(lambda self: self.info.world_size)
+    bucket_size = property(lambda self: self.info.bucket_size)
+
+    def tensor(self, t: int):
+        off, num = ctypes.c_int64(), ctypes.c_int64()
+        _check(lib.zero_plan_tensor(self._h, t, ctypes.byref(off), ctypes.byref(num)))
+        return off.value, num.value
+
+    def bucket(self, b: int):
+        s, ln = ctypes.c_int64(), ctypes.c_int64()
+        _check(lib.zero_plan_bucket(self._h, b, ctypes.byref(s), ctypes.byref(ln)))
+        return s.value, ln.value
+
+    def work_segments(self) -> List[tuple]:
+        cnt = ctypes.c_int64()
+        _check(lib.zero_plan_work_segments(self._h, None, 0, ctypes.byref(cnt)))
+        arr = (WorkSegment * max(cnt.value, 1))()
+        _check(lib.zero_plan_work_segments(self._h, arr, cnt.value, ctypes.byref(cnt)))
+        return [(s.bucket, s.rank, s.start, s.length) for s in arr[:cnt.value]]
+
+    def partition(self, rank: int) -> List[tuple]:
+        cnt = ctypes.c_int64()
+        _check(lib.zero_plan_partition(self._h, rank, None, 0, ctypes.byref(cnt)))
+        arr = (Segment * max(cnt.value, 1))()
+        _check(lib.zero_plan_partition(self._h, rank, arr, cnt.value, ctypes.byref(cnt)))
+        return [(s.tensor, s.offset_in_tensor, s.flat_offset, s.length) for s in arr[:cnt.value]]
+
+    def memory(self, stage: int) -> dict:
+        m = Memory()
+        _check(lib.zero_plan_memory(self._h, stage, ctypes.byref(m)))
+        return {f: getattr(m, f) for f, _ in Memory._fields_}
+
+    def workspace_bytes(self) -> int:
+        b = ctypes.c_size_t()
+        _check(lib.zero_workspace_bytes(self._h, ctypes.byref(b)))
+        return b.value
+
+
+def zero_plan_create(shapes, world_size, reduce_bucket_size, align=128) -> Plan:
+    return Plan(shapes, world_size, reduce_bucket_size, align)
+
+
+def zero_workspace_bytes(plan: Plan) -> int:
+    return plan.workspace_bytes()
+
+
+def scaler_cfg(dynamic: bool, initial_scale_power: int = 16, loss_scale_window: int = 100,
+               hysteresis: int = 2, min_loss_scale: float = 1.0, scale_factor: float = 2.0,
+               static_scale: float = 1.0) -> ScalerCfg:
+    return ScalerCfg(int(dynamic), initial_scale_power, loss_scale_window, hysteresis,
+                     min_loss_scale, scale_factor, static_scale)
+
+
+def adamw_cfg(lr=6e-5, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01,
+              max_grad_norm=1.0) -> AdamWCfg:
+    return AdamWCfg(lr, beta1, beta2, eps, weight_decay, max_grad_norm)
+
+
+# ---------------------------------------------------------------------------- the step
+
+def zero_state_init(plan: Plan, workspace, cfg: ScalerCfg, stream=None) -> None:
+    _check(lib.zero_state_init(plan.handle, _addr(workspace), ctypes.byref(cfg), _stream(stream)))
+
+
+def zero_cast_params(plan: Plan, master, params, param_dtype, stream=None) -> None:
+    _check(lib.zero_cast_params(plan.handle, _addr(master), _addr(params), _dtype(param_dtype),
+                                _stream(stream)))
+
+
+def zero_reduce_scatter_bucket(plan: Plan, bucket: int, grad_dtype, replica_grads: Sequence,
+                               replica_base_offset: int, reduced, workspace, stream=None) -> None:
+    _check(lib.zero_reduce_scatter_bucket(plan.handle, bucket, _dtype(grad_dtype),
+                                          _ptr_array(replica_grads), int(replica_base_offset),
+                                          _addr(reduced), _addr(workspace), _stream(stream)))
+
+
+def zero_reduce_scatter_bucket_host(plan: Plan, bucket: int, grad_dtype,
+                                    host_replica_grads: Sequence, host_base_offset: int,
+                                    device_staging: Sequence, reduced, workspace,
+                                    stream=None) -> None:
+    _check(lib.zero_reduce_scatter_bucket_host(
+        plan.handle, bucket, _dtype(grad_dtype), _ptr_array(host_replica_grads),
+        int(host_base_offset), _ptr_array(device_staging), _addr(reduced), _addr(workspace),
+        _stream(stream)))
+
+
+def zero_step(plan: Plan, cfg: AdamWCfg, master, exp_avg, exp_avg_sq, reduced, params,
+              param_dtype, workspace, stream=None) -> None:
+    _check(lib.zero_step(plan.handle, ctypes.byref(cfg), _addr(master), _addr(exp_avg),
+                         _addr(exp_avg_sq), _addr(reduced), _addr(params), _dtype(param_dtype),
+                         _addr(workspace), _stream(stream)))
+
+
+def zero_step_finalize(plan: Plan, cfg: AdamWCfg, workspace, stream=None) -> None:
+    _check(lib.zero_step_finalize(plan.handle, ctypes.byref(cfg), _addr(workspace),
+                                  _stream(stream)))
+
+
+def zero_step_update(plan: Plan, master, exp_avg, exp_avg_sq, reduced, params, param_dtype,
+                     workspace, stream=None) -> None:
+    _check(lib.zero_step_update(plan.handle, _addr(master), _addr(exp_avg), _addr(exp_avg_sq),
+                                _addr(reduced), _addr(params), _dtype(param_dtype),
+                                _addr(workspace), _stream(stream)))
+
+
+def zero_all_gather(plan: Plan, params, rank_params: Sequence, param_dtype, stream=None) -> None:
+    arr = _ptr_array(rank_params) if rank_params else None
+    _check(lib.zero_all_gather(plan.handle, _addr(params), arr, len(rank_params),
+                               _dtype(param_dtype), _stream(stream)))
+
+
+def zero_get_result(workspace, stream=None) -> dict:
+    r = StepResult()
+    _check(lib.zero_get_result(_addr(workspace), ctypes.byref(r), _stream(stream)))
+    return r.as_dict()
+
+
+def zero_abi_version() -> int:
+    return lib.zero_abi_version()
+
+
+from .optimizer import ZeroOptimizer  # noqa: E402  (torch plumbing around the calls above)

@@ -1,0 +1,88 @@
+"""ZeroOptimizer: device buffers for one ZeRO partitioned optimizer (torch allocates them,
+the library's kernels do all the work).
+
+Buffers, all flat over the padded parameter space of the plan (n_pad elements):
+  master, exp_avg, exp_avg_sq  fp32   rank r owns [r*p, (r+1)*p) of each
+  reduced                      fp32   reduce-scattered gradient, same ownership
+  params                       half   the gathered parameter buffer
+  workspace                    bytes  scaler state, partial sums, step result
+"""
+from __future__ import annotations
+
+from typing import Optional, Sequence
+
+import torch
+
+from . import (AdamWCfg, Plan, ScalerCfg, adamw_cfg, scaler_cfg, zero_all_gather,
+               zero_cast_params, zero_get_result, zero_reduce_scatter_bucket,
+               zero_reduce_scatter_bucket_host, zero_state_init, zero_step,
+               zero_step_finalize, zero_step_update)
+
+_TORCH_HALF = {"bf16": torch.bfloat16, "fp16": torch.float16}
+
+
+class ZeroOptimizer:
+    def __init__(self, shapes: Sequence[Sequence[int]], world_size: int,
+                 reduce_bucket_size: int, dtype: str = "bf16", align: int = 128,
+                 scaler: Optional[ScalerCfg] = None, adamw: Optional[AdamWCfg] = None,
+                 device: str = "cuda", stream: Optional[torch.cuda.Stream] = None):
+        self.plan = Plan(shapes, world_size, reduce_bucket_size, align)
+        self.dtype = dtype
+        self.device = torch.device(device)
+        self.stream = stream
+        n = self.plan.n_pad
+        f32 = dict(dtype=torch.float32, device=self.device)
+        self.master = torch.zeros(n, **f32)
+        self.exp_avg = torch.zeros(n, **f32)
+        self.exp_avg_sq = torch.zeros(n, **f32)
+        self.reduced = torch.zeros(n, **f32)
+        self.params = torch.zeros(n, dtype=_TORCH_HALF[dtype], device=self.device)
+        self.workspace = torch.zeros(self.plan.workspace_bytes(), dtype=torch.uint8,
+                                     device=self.device)
+        self.scaler = scaler if scaler is not None else scaler_cfg(dynamic=(dtype == "fp16"))
+        self.adamw = adamw if adamw is not None else adamw_cfg()
+        zero_state_init(self.plan, self.workspace, self.scaler, self._s())
+
+    def _s(self):
+        return self.stream.cuda_stream if self.stream is not None else \
+            torch.cuda.current_stream(self.device).cuda_stream
+
+    # -------------------------------------------------------------- step pieces
+    def cast_params(self) -> None:
+        """params <- round_to_nearest_even(master): after initialising or loading master."""
+        zero_cast_params(self.plan, self.master, self.params, self.dtype, self._s())
+
+    def reduce_scatter_bucket(self, bucket: int, replica_grads: Sequence, base_offset: int = 0):
+        zero_reduce_scatter_bucket(self.plan, bucket, self.dtype, replica_grads, base_offset,
+                                   self.reduced, self.workspace, self._s())
+
+    def reduce_scatter_bucket_host(self, bucket: int, host_replica_grads: Sequence,
+                                   host_base_offset: int, device_staging: Sequence):
+        zero_reduce_scatter_bucket_host(self.plan, bucket, self.dtype, host_replica_grads,
+                                        host_base_offset, device_staging, self.reduced,
+                                        self.workspace, self._s())
+
+    def step(self) -> None:
+        zero_step(self.plan, self.adamw, self.master, self.exp_avg, self.exp_avg_sq,
+                  self.reduced, self.params, self.dtype, self.workspace, self._s())
+
+    def step_finalize(self) -> None:
+        zero_step_finalize(self.plan, self.adamw, self.workspace, self._s())
+
+    def step_update(self) -> None:
+        zero_step_update(self.plan, self.master, self.exp_avg, self.exp_avg_sq, self.reduced,
+                         self.params, self.dtype, self.workspace, self._s())
+
+    def all_gather(self, rank_params: Sequence = ()) -> None:
+        zero_all_gather(self.plan, self.params, list(rank_params), self.dtype, self._s())
+
+    def result(self) -> dict:
+        """Step result; synchronises the stream."""
+        return zero_get_result(self.workspace, self._s())
+
+    # -------------------------------------------------------------- whole step
+    def full_step(self, replica_grads: Sequence, base_offset: int = 0) -> None:
+        """Reduce-scatter every bucket from whole-model replica buffers, then step."""
+        for b in range(self.plan.n_buckets):
+            self.reduce_scatter_bucket(b, replica_grads, base_offset)
+        self.step()
