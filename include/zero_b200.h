@@ -254,6 +254,34 @@ ZERO_API int zero_all_gather(const zero_plan* plan, const void* params, void* co
 /* Copies the step result out of the workspace and synchronises `stream`. */
 ZERO_API int zero_get_result(const void* workspace, zero_step_result* out, void* stream);
 
+/* ---------------------------------------------------------------- no-alloc variant
+ * zero_reduce_sumsq_noalloc has no counterpart in the pages. It is for callers that
+ * cannot allocate device memory for a workspace: for example a C plugin that its host
+ * framework hands only the input and output buffers, with no access to that
+ * framework's allocator, or a loop that must not call cudaMalloc because cudaMalloc can
+ * synchronise the whole device.
+ * Without a plan or a workspace it computes what zero_reduce_scatter_bucket computes for
+ * one bucket:
+ *   reduced[i] = ((g_0[i] + g_1[i]) + ...) + g_{W-1}[i]   (fp32, rank order), i < n,
+ * and writes the fp64 sum of squares of reduced[0 .. n) to *sumsq (device memory).
+ * Scratch: the per-block partial sums go to an array of ZERO_NOALLOC_MAX_BLOCKS fp64
+ * slots (512 KB) compiled into the library; every GPU that loads the library holds it
+ * until the process exits. One block covers 2048 elements, so n may be at most
+ * ZERO_NOALLOC_MAX_ELEMS; a larger n returns ZERO_ERANGE (split the range into calls).
+ * The first call on a device looks up the array's device address with that device
+ * current; make that first call before any stream capture.
+ * Every call uses the same array and writes each slot before reading it, so nothing
+ * needs clearing between calls; calls that overlap on the GPU (other streams, other
+ * host threads) race on the array and return wrong sums, so serialise them.
+ * replica_grads is a HOST array of world_size device pointers (16-byte aligned);
+ * reduced must be 16-byte aligned and sumsq 8-byte aligned. Errors: EINVAL (W outside
+ * [1, 16], bad dtype, NULL pointer, n < 0), EALIGN, ERANGE (n too large), ECUDA. */
+#define ZERO_NOALLOC_MAX_BLOCKS 65536
+#define ZERO_NOALLOC_MAX_ELEMS ((int64_t)ZERO_NOALLOC_MAX_BLOCKS * 2048)
+ZERO_API int zero_reduce_sumsq_noalloc(int32_t world_size, int32_t grad_dtype,
+                                       const void* const* replica_grads, int64_t n,
+                                       float* reduced, double* sumsq, void* stream);
+
 ZERO_API const char* zero_last_error(void);
 ZERO_API int zero_abi_version(void);
 
