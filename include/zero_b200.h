@@ -69,6 +69,8 @@ extern "C" {
 #define ZERO_ESTATE (-4) /* call out of order: a bucket reduced twice, or a step before every bucket was reduced */
 #define ZERO_ECUDA (-5)  /* a CUDA launch or copy failed; the message names the CUDA error */
 #define ZERO_ENOMEM (-6) /* host allocation for the plan failed */
+#define ZERO_EDEVICE (-7) /* a kernel gave up waiting on its own pipeline (bounded waits of
+                             about one second); its output is incomplete */
 
 /* element types of gradients and gathered parameters */
 #define ZERO_BF16 0
@@ -132,7 +134,8 @@ typedef struct {
   int32_t overflow;   /* a reduced gradient was inf or NaN                           */
   int32_t skipped;    /* the update was skipped (overflow)                           */
   int32_t hysteresis; /* hysteresis budget after the step                            */
-  int32_t reserved;
+  int32_t device_error; /* nonzero once a kernel gave up on a bounded wait (sticky until
+                           zero_state_init); zero_get_result then returns ZERO_EDEVICE */
   int64_t iter;       /* scaler iterations so far (every step)                       */
   int64_t adam_t;     /* applied AdamW steps so far                                  */
 } zero_step_result;
@@ -251,7 +254,8 @@ ZERO_API int zero_step_update(zero_plan* plan, float* master, float* exp_avg, fl
 ZERO_API int zero_all_gather(const zero_plan* plan, const void* params, void* const* rank_params,
                     int32_t n_dst, int32_t param_dtype, void* stream);
 
-/* Copies the step result out of the workspace and synchronises `stream`. */
+/* Copies the step result out of the workspace and synchronises `stream`. Returns
+ * ZERO_EDEVICE (with *out filled) if a kernel reported a timed-out internal wait. */
 ZERO_API int zero_get_result(const void* workspace, zero_step_result* out, void* stream);
 
 /* ---------------------------------------------------------------- no-alloc variant

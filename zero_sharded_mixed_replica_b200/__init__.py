@@ -27,13 +27,15 @@ ZERO_ERANGE = -3
 ZERO_ESTATE = -4
 ZERO_ECUDA = -5
 ZERO_ENOMEM = -6
+ZERO_EDEVICE = -7
 ZERO_BF16 = 0
 ZERO_FP16 = 1
 ZERO_MAX_WORLD = 16
 DTYPES = {"bf16": ZERO_BF16, "fp16": ZERO_FP16}
 
 _ERR_NAMES = {ZERO_EINVAL: "EINVAL", ZERO_EALIGN: "EALIGN", ZERO_ERANGE: "ERANGE",
-              ZERO_ESTATE: "ESTATE", ZERO_ECUDA: "ECUDA", ZERO_ENOMEM: "ENOMEM"}
+              ZERO_ESTATE: "ESTATE", ZERO_ECUDA: "ECUDA", ZERO_ENOMEM: "ENOMEM",
+              ZERO_EDEVICE: "EDEVICE"}
 
 
 class ZeroError(RuntimeError):
@@ -78,11 +80,11 @@ class StepResult(ctypes.Structure):
                 ("clip_coef", ctypes.c_float), ("scale_used", ctypes.c_float),
                 ("next_scale", ctypes.c_float), ("k", ctypes.c_float),
                 ("overflow", ctypes.c_int32), ("skipped", ctypes.c_int32),
-                ("hysteresis", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("hysteresis", ctypes.c_int32), ("device_error", ctypes.c_int32),
                 ("iter", ctypes.c_int64), ("adam_t", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
-        return {f: getattr(self, f) for f, _ in self._fields_ if f != "reserved"}
+        return {f: getattr(self, f) for f, _ in self._fields_}
 
 
 class Memory(ctypes.Structure):

@@ -59,9 +59,10 @@ int reduce_bucket(zero_plan* plan, int64_t b, int32_t dt, const uint16_t* const*
   int grid = 1;
   cudaError_t e = rs_grid(len, plan->world, dt, &grid);
   if (e != cudaSuccess) return cuda_fail(e, "reduce-scatter occupancy query");
-  e = launch_reduce_scatter(plan->world, dt, g_at_start, reduced + start, start, len,
+  e = launch_reduce_scatter(plan->world, dt, g_at_start, reduced + start, len,
                             ws_partial(plan, ws) + b * plan->slots_full,
-                            ws_bucket_blocks(plan, ws) + b, grid, s);
+                            ws_bucket_blocks(plan, ws) + b,
+                            &((WsHeader*)ws)->result.device_error, grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "reduce-scatter launch");
   plan->reduced[b] = 1;
   plan->reduced_count += 1;
@@ -455,6 +456,9 @@ int zero_get_result(const void* workspace, zero_step_result* out, void* stream) 
   if (e != cudaSuccess) return cuda_fail(e, "result copy");
   e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  if (out->device_error)
+    return fail(ZERO_EDEVICE, "a kernel gave up on a bounded internal wait (code " +
+                                  std::to_string(out->device_error) + "); outputs are incomplete");
   return ZERO_OK;
 }
 

@@ -37,15 +37,6 @@ __device__ __forceinline__ float4 ld_nc_f4(const float* p) {
   return r;
 }
 
-// coherent load for data this kernel later overwrites at the same address
-__device__ __forceinline__ float4 ld_f4(const float* p) {
-  float4 r;
-  asm("ld.global.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
-      : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
-      : "l"(p));
-  return r;
-}
-
 __device__ __forceinline__ void st_f4(float* p, float a, float b, float c, float d) {
   asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
                "f"(d)
@@ -56,6 +47,77 @@ __device__ __forceinline__ void st_u4(void* p, uint32_t a, uint32_t b, uint32_t 
   asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c),
                "r"(d)
                : "memory");
+}
+
+__device__ __forceinline__ void st_cs_f4(float* p, float a, float b, float c, float d) {
+  asm volatile("st.global.cs.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+// ------------------------------------------------------------------ TMA bulk copies
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// arrive and announce `bytes` of bulk copies that will complete on this barrier phase
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for the phase with the given parity to complete, at most about one second;
+// false when the wait gave up.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  return true;
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar` (addresses and
+// size multiples of 16 bytes). No multicast.
+__device__ __forceinline__ void bulk_load(void* dst_smem, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst_smem)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
 }
 
 // ------------------------------------------------------------------ half helpers
@@ -136,80 +198,164 @@ struct RsArgs {
   int64_t len;                        // elements in the bucket
   int64_t head;                       // scalar elements before the first aligned group
   int64_t nvec;                       // aligned groups of 8 elements
+  int32_t* device_error;              // sticky error word, or null
 };
+
+// Pipeline shape of the reduce-scatter: each of kRsStages shared-memory stages holds the
+// W replica tiles of one tile (rs_tile<W>() halves each, about 64 KB per stage); one
+// producer thread keeps the stages filled with 1-D bulk copies, kRsConsumers threads sum
+// from shared memory. One CTA per SM.
+constexpr int kRsStages = 3;
+constexpr int kRsConsumers = 256;
+constexpr int kRsTmaThreads = kRsConsumers + 32;
+
+template <int W>
+__host__ __device__ constexpr int rs_tile() {
+  // a multiple of 2048 (one 8-element group per consumer thread) near 32768 / W
+  return (32768 / W) / 2048 * 2048 < 2048 ? 2048 : (32768 / W) / 2048 * 2048;
+}
+
+template <int W>
+__host__ __device__ constexpr size_t rs_smem_bytes() {
+  return (size_t)kRsStages * W * rs_tile<W>() * sizeof(uint16_t) + 2 * kRsStages * sizeof(uint64_t);
+}
 
 // For every element i of the bucket: R[i] = ((g_0[i] + g_1[i]) + ...) + g_{W-1}[i] in
 // fp32, and ss += R[i]^2 in fp64 (the square of an fp32 is exact in fp64, so the fused
-// multiply-add rounds exactly like the separate add would). Each block writes its ss
-// to its own slot; the finalize kernel adds the slots in a fixed order.
-// U groups per thread per trip keep >= 8 16-byte loads in flight for small W.
-template <int W, int DT, int U>
-__global__ void __launch_bounds__(kRsThreads) rs_bucket_kernel(const __grid_constant__ RsArgs a) {
-  double ss = 0.0;
-  const int64_t nthr = (int64_t)gridDim.x * kRsThreads;
-  const int64_t tid = (int64_t)blockIdx.x * kRsThreads + threadIdx.x;
-  for (int64_t v0 = tid; v0 < a.nvec; v0 += nthr * U) {
-    uint4 x[U][W];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t v = v0 + (int64_t)u * nthr;
-      if (v < a.nvec) {
-        const int64_t e = a.head + v * 8;
-#pragma unroll
-        for (int r = 0; r < W; ++r) x[u][r] = ld_nc_u4(a.g[r] + e);
-      }
+// multiply-add rounds exactly like the separate add would). Full tiles of the aligned
+// body [head, head + 8*nvec) go through the TMA pipeline; the last CTA takes the rest
+// (the unaligned head, the groups after the last full tile, the last < 8 elements).
+// Each CTA writes its ss to its own slot; the finalize kernel adds the slots in a fixed
+// order. A wait that gives up (about one second) ends the CTA's pipeline early and
+// records a code in *device_error when that pointer is set.
+template <int W, int DT>
+__global__ void __launch_bounds__(kRsTmaThreads, 1)
+    rs_bucket_kernel(const __grid_constant__ RsArgs a) {
+  constexpr int TILE = rs_tile<W>();
+  constexpr uint32_t kStageBytes = (uint32_t)W * TILE * sizeof(uint16_t);
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint16_t* stage_buf = (uint16_t*)smem;  // [kRsStages][W][TILE]
+  uint64_t* full = (uint64_t*)(smem + (size_t)kRsStages * kStageBytes);
+  uint64_t* empty = full + kRsStages;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    for (int st = 0; st < kRsStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], kRsConsumers / 32);
     }
+    mbar_init_fence();
+  }
+  __syncthreads();
+
+  const int64_t n_tiles = (8 * a.nvec) / TILE;
+  const int64_t G = gridDim.x;
+  double ss = 0.0;
+
+  if (tid >= kRsConsumers) {
+    if (tid == kRsConsumers) {  // producer
+      int64_t k = 0;
+      for (int64_t t = blockIdx.x; t < n_tiles; t += G, ++k) {
+        const int st = (int)(k % kRsStages);
+        if (k >= kRsStages && !mbar_wait(&empty[st], (uint32_t)((k / kRsStages - 1) & 1))) {
+          if (a.device_error) atomicOr(a.device_error, 8);
+          break;
+        }
+        mbar_arrive_expect_tx(&full[st], kStageBytes);
+        uint16_t* dst = stage_buf + (size_t)st * W * TILE;
+        const int64_t off = a.head + t * TILE;
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t v = v0 + (int64_t)u * nthr;
-      if (v < a.nvec) {
-        const int64_t e = a.head + v * 8;
+        for (int r = 0; r < W; ++r)
+          bulk_load(dst + r * TILE, a.g[r] + off, TILE * sizeof(uint16_t), &full[st]);
+      }
+      for (int64_t j = k > kRsStages ? k - kRsStages : 0; j < k; ++j)
+        if (!mbar_wait(&full[j % kRsStages], (uint32_t)((j / kRsStages) & 1)) && a.device_error)
+          atomicOr(a.device_error, 32);
+    }
+  } else {
+    int64_t k = 0;
+    for (int64_t t = blockIdx.x; t < n_tiles; t += G, ++k) {
+      const int st = (int)(k % kRsStages);
+      if (!mbar_wait(&full[st], (uint32_t)((k / kRsStages) & 1))) {
+        if (a.device_error) atomicOr(a.device_error, 16);
+        break;
+      }
+      const uint16_t* src = stage_buf + (size_t)st * W * TILE;
+      const int64_t off = a.head + t * TILE;
+#pragma unroll
+      for (int q = 0; q < TILE / (8 * kRsConsumers); ++q) {
+        const int e = (q * kRsConsumers + tid) * 8;
         float acc[8];
-        unpack8<DT>(x[u][0], acc);
+        unpack8<DT>(*(const uint4*)(src + e), acc);
 #pragma unroll
         for (int r = 1; r < W; ++r) {
-          float t[8];
-          unpack8<DT>(x[u][r], t);
+          float x[8];
+          unpack8<DT>(*(const uint4*)(src + r * TILE + e), x);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[j] = __fadd_rn(acc[j], t[j]);
+          for (int j = 0; j < 8; ++j) acc[j] = __fadd_rn(acc[j], x[j]);
         }
-        st_f4(a.R + e, acc[0], acc[1], acc[2], acc[3]);
-        st_f4(a.R + e + 4, acc[4], acc[5], acc[6], acc[7]);
+        // R is read back only after every bucket of the step: stream it past the caches
+        st_cs_f4(a.R + off + e, acc[0], acc[1], acc[2], acc[3]);
+        st_cs_f4(a.R + off + e + 4, acc[4], acc[5], acc[6], acc[7]);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const double d = (double)acc[j];
           ss = __fma_rn(d, d, ss);
         }
       }
+      __syncwarp();
+      if ((tid & 31) == 0) mbar_arrive(&empty[st]);
+    }
+
+    if (blockIdx.x == G - 1) {
+      // aligned groups after the last full tile, with plain 16-byte loads
+      const int64_t vec_end = a.head + 8 * a.nvec;
+      for (int64_t e = a.head + n_tiles * TILE + 8 * (int64_t)tid; e < vec_end;
+           e += 8 * kRsConsumers) {
+        float acc[8];
+        unpack8<DT>(ld_nc_u4(a.g[0] + e), acc);
+#pragma unroll
+        for (int r = 1; r < W; ++r) {
+          float x[8];
+          unpack8<DT>(ld_nc_u4(a.g[r] + e), x);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[j] = __fadd_rn(acc[j], x[j]);
+        }
+        st_cs_f4(a.R + e, acc[0], acc[1], acc[2], acc[3]);
+        st_cs_f4(a.R + e + 4, acc[4], acc[5], acc[6], acc[7]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const double d = (double)acc[j];
+          ss = __fma_rn(d, d, ss);
+        }
+      }
+      // scalar elements: the unaligned head [0, head) and the last (len - vec_end)
+      const int64_t n_scalar = a.head + (a.len - vec_end);
+      for (int64_t q = tid; q < n_scalar; q += kRsConsumers) {
+        const int64_t i = q < a.head ? q : vec_end + (q - a.head);
+        float acc = half_bits_to_float<DT>(a.g[0][i]);
+#pragma unroll
+        for (int r = 1; r < W; ++r) acc = __fadd_rn(acc, half_bits_to_float<DT>(a.g[r][i]));
+        a.R[i] = acc;
+        const double d = (double)acc;
+        ss = __fma_rn(d, d, ss);
+      }
     }
   }
-  // scalar elements: the unaligned head [0, head) and the tail after the last group
-  const int64_t body_end = a.head + 8 * a.nvec;
-  const int64_t n_scalar = a.head + (a.len - body_end);
-  for (int64_t q = tid; q < n_scalar; q += nthr) {
-    const int64_t i = q < a.head ? q : body_end + (q - a.head);
-    float acc = half_bits_to_float<DT>(a.g[0][i]);
-#pragma unroll
-    for (int r = 1; r < W; ++r) acc = __fadd_rn(acc, half_bits_to_float<DT>(a.g[r][i]));
-    a.R[i] = acc;
-    const double d = (double)acc;
-    ss = __fma_rn(d, d, ss);
-  }
-  ss = block_sum<kRsThreads>(ss);
-  if (threadIdx.x == 0) {
+  ss = block_sum<kRsTmaThreads>(ss);
+  if (tid == 0) {
     a.partial[blockIdx.x] = ss;
     if (blockIdx.x == 0) *a.blocks = (int32_t)gridDim.x;
   }
 }
 
 template <int W, int DT>
-constexpr int rs_unroll() {
-  return W >= 8 ? 1 : (W >= 4 ? 2 : 4);
+const void* rs_kernel_ptr() {
+  return (const void*)rs_bucket_kernel<W, DT>;
 }
 
-template <int W, int DT>
-const void* rs_kernel_ptr() {
-  return (const void*)rs_bucket_kernel<W, DT, rs_unroll<W, DT>()>;
+template <int W>
+size_t rs_smem_for() {
+  return rs_smem_bytes<W>();
 }
 
 typedef const void* (*KernelGetter)();
@@ -220,13 +366,20 @@ struct RsTable {
     const void* ptrs[] = {rs_kernel_ptr<Ws, DT>()...};
     return ptrs[w - 1];
   }
+  static size_t smem(int w) {
+    const size_t bytes[] = {rs_smem_for<Ws>()...};
+    return bytes[w - 1];
+  }
 };
 
+using RsBf16 = RsTable<ZERO_BF16, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15, 16>;
+using RsFp16 = RsTable<ZERO_FP16, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15, 16>;
+
 const void* rs_kernel_for(int world, int dtype) {
-  if (dtype == ZERO_BF16)
-    return RsTable<ZERO_BF16, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15, 16>::get(world);
-  return RsTable<ZERO_FP16, 1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 14, 15, 16>::get(world);
+  return dtype == ZERO_BF16 ? RsBf16::get(world) : RsFp16::get(world);
 }
+
+size_t rs_smem_for_world(int world) { return RsBf16::smem(world); }
 
 // ================================================================== K2: finalize
 
@@ -306,9 +459,8 @@ __global__ void __launch_bounds__(kFinalizeThreads)
   r.overflow = overflow;
   r.skipped = overflow;
   r.hysteresis = h->cur_hysteresis;
-  r.reserved = 0;
   r.iter = h->iter;
-  r.adam_t = t;
+  r.adam_t = t;  // r.device_error is left as it is: sticky until zero_state_init
 }
 
 // ================================================================== K3: AdamW + cast
@@ -321,6 +473,7 @@ struct UpArgs {
   void* out;  // gathered half buffer
   int64_t n;
   const WsHeader* h;
+  int32_t* device_error;  // &h->result.device_error
 };
 
 struct AdamConsts {
@@ -338,8 +491,24 @@ __device__ __forceinline__ void adamw1(const AdamConsts& c, float r, float& p, f
   p = __fsub_rn(__fmul_rn(p, c.decay), __fmul_rn(c.lr, __fdiv_rn(t1, t2)));
 }
 
+// Pipeline shape: tiles of kUpTile elements; each of kUpStages shared-memory stages holds
+// the R, p, m, v tiles (4 x 16 KB); one producer thread keeps the stages filled with
+// 1-D bulk copies while kUpConsumers threads compute from shared memory and store the
+// results straight to global memory. One CTA per SM (about 192 KB of shared memory).
+constexpr int kUpTile = 4096;
+constexpr int kUpStages = 3;
+constexpr int kUpConsumers = 256;
+constexpr int kUpTmaThreads = kUpConsumers + 32;  // + one producer warp
+constexpr size_t kUpStageBytes = 4ull * kUpTile * sizeof(float);
+constexpr size_t kUpSmemBytes = kUpStages * kUpStageBytes + 2 * kUpStages * sizeof(uint64_t);
+
+// AdamW + half cast over [0, n): full tiles through the TMA pipeline, the last
+// n % kUpTile elements by the last CTA with plain loads. Returns at once (every thread)
+// when the finalize step decided to skip. A wait that gives up (about one second)
+// records a code in *device_error and ends the CTA's work early.
 template <int DT>
-__global__ void __launch_bounds__(kUpThreads) adamw_cast_kernel(const __grid_constant__ UpArgs a) {
+__global__ void __launch_bounds__(kUpTmaThreads, 1)
+    adamw_cast_kernel(const __grid_constant__ UpArgs a) {
   const WsHeader* h = a.h;
   if (h->skip) return;  // overflow: the whole step is skipped
   AdamConsts c;
@@ -353,40 +522,93 @@ __global__ void __launch_bounds__(kUpThreads) adamw_cast_kernel(const __grid_con
   c.eps = h->eps;
   c.lr = h->lr;
   c.decay = h->decay;
-  const int64_t nthr = (int64_t)gridDim.x * kUpThreads;
-  const int64_t tid = (int64_t)blockIdx.x * kUpThreads + threadIdx.x;
-  const int64_t nvec = a.n / 8;
-  uint16_t* out = (uint16_t*)a.out;
-  for (int64_t vi = tid; vi < nvec; vi += nthr) {
-    const int64_t e = vi * 8;
-    const float4 r0 = ld_nc_f4(a.R + e), r1 = ld_nc_f4(a.R + e + 4);
-    float4 p0 = ld_f4(a.p + e), p1 = ld_f4(a.p + e + 4);
-    float4 m0 = ld_f4(a.m + e), m1 = ld_f4(a.m + e + 4);
-    float4 v0 = ld_f4(a.v + e), v1 = ld_f4(a.v + e + 4);
-    adamw1(c, r0.x, p0.x, m0.x, v0.x);
-    adamw1(c, r0.y, p0.y, m0.y, v0.y);
-    adamw1(c, r0.z, p0.z, m0.z, v0.z);
-    adamw1(c, r0.w, p0.w, m0.w, v0.w);
-    adamw1(c, r1.x, p1.x, m1.x, v1.x);
-    adamw1(c, r1.y, p1.y, m1.y, v1.y);
-    adamw1(c, r1.z, p1.z, m1.z, v1.z);
-    adamw1(c, r1.w, p1.w, m1.w, v1.w);
-    st_f4(a.p + e, p0.x, p0.y, p0.z, p0.w);
-    st_f4(a.p + e + 4, p1.x, p1.y, p1.z, p1.w);
-    st_f4(a.m + e, m0.x, m0.y, m0.z, m0.w);
-    st_f4(a.m + e + 4, m1.x, m1.y, m1.z, m1.w);
-    st_f4(a.v + e, v0.x, v0.y, v0.z, v0.w);
-    st_f4(a.v + e + 4, v1.x, v1.y, v1.z, v1.w);
-    st_u4(out + e, pack2<DT>(p0.x, p0.y), pack2<DT>(p0.z, p0.w), pack2<DT>(p1.x, p1.y),
-          pack2<DT>(p1.z, p1.w));
+
+  extern __shared__ __align__(128) unsigned char smem[];
+  float* stage_buf = (float*)smem;  // [kUpStages][R, p, m, v][kUpTile]
+  uint64_t* full = (uint64_t*)(smem + kUpStages * kUpStageBytes);
+  uint64_t* empty = full + kUpStages;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    for (int st = 0; st < kUpStages; ++st) {
+      mbar_init(&full[st], 1);                   // the producer's expect_tx arrival
+      mbar_init(&empty[st], kUpConsumers / 32);  // one arrival per consumer warp
+    }
+    mbar_init_fence();
   }
-  for (int64_t i = nvec * 8 + tid; i < a.n; i += nthr) {
-    float p = a.p[i], m = a.m[i], v = a.v[i];
-    adamw1(c, a.R[i], p, m, v);
-    a.p[i] = p;
-    a.m[i] = m;
-    a.v[i] = v;
-    out[i] = (uint16_t)float_to_half_bits<DT>(p);
+  __syncthreads();
+
+  const int64_t n_tiles = a.n / kUpTile;
+  const int64_t G = gridDim.x;
+  uint16_t* out = (uint16_t*)a.out;
+
+  if (tid >= kUpConsumers) {
+    // producer warp: one thread issues the bulk copies
+    if (tid == kUpConsumers) {
+      int64_t k = 0;
+      for (int64_t t = blockIdx.x; t < n_tiles; t += G, ++k) {
+        const int st = (int)(k % kUpStages);
+        if (k >= kUpStages &&
+            !mbar_wait(&empty[st], (uint32_t)((k / kUpStages - 1) & 1))) {
+          atomicOr(a.device_error, 1);
+          break;
+        }
+        if (*(volatile int32_t*)a.device_error) break;
+        mbar_arrive_expect_tx(&full[st], (uint32_t)kUpStageBytes);
+        const int64_t off = t * kUpTile;
+        float* dst = stage_buf + (size_t)st * 4 * kUpTile;
+        bulk_load(dst, a.R + off, kUpTile * 4, &full[st]);
+        bulk_load(dst + kUpTile, a.p + off, kUpTile * 4, &full[st]);
+        bulk_load(dst + 2 * kUpTile, a.m + off, kUpTile * 4, &full[st]);
+        bulk_load(dst + 3 * kUpTile, a.v + off, kUpTile * 4, &full[st]);
+      }
+      // before the CTA exits: the copies of the last stages must have landed
+      for (int64_t j = k > kUpStages ? k - kUpStages : 0; j < k; ++j)
+        if (!mbar_wait(&full[j % kUpStages], (uint32_t)((j / kUpStages) & 1)))
+          atomicOr(a.device_error, 4);
+    }
+    return;
+  }
+
+  // consumers: each thread takes 4 consecutive elements per 1024-element slice
+  int64_t k = 0;
+  for (int64_t t = blockIdx.x; t < n_tiles; t += G, ++k) {
+    const int st = (int)(k % kUpStages);
+    if (!mbar_wait(&full[st], (uint32_t)((k / kUpStages) & 1))) {
+      atomicOr(a.device_error, 2);
+      break;
+    }
+    const float* src = stage_buf + (size_t)st * 4 * kUpTile;
+    const int64_t off = t * kUpTile;
+#pragma unroll
+    for (int q = 0; q < kUpTile / (4 * kUpConsumers); ++q) {
+      const int e = (q * kUpConsumers + tid) * 4;
+      const float4 r = *(const float4*)(src + e);
+      float4 p = *(const float4*)(src + kUpTile + e);
+      float4 m = *(const float4*)(src + 2 * kUpTile + e);
+      float4 v = *(const float4*)(src + 3 * kUpTile + e);
+      adamw1(c, r.x, p.x, m.x, v.x);
+      adamw1(c, r.y, p.y, m.y, v.y);
+      adamw1(c, r.z, p.z, m.z, v.z);
+      adamw1(c, r.w, p.w, m.w, v.w);
+      st_f4(a.p + off + e, p.x, p.y, p.z, p.w);
+      st_f4(a.m + off + e, m.x, m.y, m.z, m.w);
+      st_f4(a.v + off + e, v.x, v.y, v.z, v.w);
+      *(uint2*)(out + off + e) = make_uint2(pack2<DT>(p.x, p.y), pack2<DT>(p.z, p.w));
+    }
+    __syncwarp();
+    if ((tid & 31) == 0) mbar_arrive(&empty[st]);
+  }
+
+  // the ragged tail after the last full tile
+  if (blockIdx.x == G - 1) {
+    for (int64_t i = n_tiles * kUpTile + tid; i < a.n; i += kUpConsumers) {
+      float p = a.p[i], m = a.m[i], v = a.v[i];
+      adamw1(c, a.R[i], p, m, v);
+      a.p[i] = p;
+      a.m[i] = m;
+      a.v[i] = v;
+      out[i] = (uint16_t)float_to_half_bits<DT>(p);
+    }
   }
 }
 
@@ -453,7 +675,7 @@ __global__ void state_init_kernel(WsHeader* h, zero_scaler_cfg cfg) {
   r.overflow = 0;
   r.skipped = 0;
   r.hysteresis = h->cur_hysteresis;
-  r.reserved = 0;
+  r.device_error = 0;
   r.iter = 0;
   r.adam_t = 0;
 }
@@ -499,14 +721,18 @@ int64_t rs_slots(int64_t len) {
 }
 
 cudaError_t rs_grid(int64_t len, int world, int dtype, int* grid) {
+  const void* k = rs_kernel_for(world, dtype);
+  const size_t smem = rs_smem_for_world(world);
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   int per_sm = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-      &per_sm, rs_kernel_for(world, dtype), kRsThreads, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kRsTmaThreads, smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
   int64_t g = (int64_t)per_sm * sm_count();
   const int64_t cap = rs_slots(len);
   if (g > cap) g = cap;
+  if (g < 1) g = 1;
   *grid = (int)g;
   return cudaSuccess;
 }
@@ -517,9 +743,10 @@ cudaError_t launch_state_init(void* ws, const zero_scaler_cfg& cfg, cudaStream_t
 }
 
 cudaError_t launch_reduce_scatter(int world, int dtype, const uint16_t* const* g, float* R,
-                                  int64_t /*start*/, int64_t len, double* partial,
-                                  int32_t* bucket_blocks, int grid, cudaStream_t s) {
+                                  int64_t len, double* partial, int32_t* bucket_blocks,
+                                  int32_t* device_error, int grid, cudaStream_t s) {
   RsArgs a;
+  a.device_error = device_error;
   for (int r = 0; r < ZERO_MAX_WORLD; ++r) a.g[r] = r < world ? g[r] : nullptr;
   a.R = R;
   a.partial = partial;
@@ -554,8 +781,12 @@ cudaError_t launch_reduce_scatter(int world, int dtype, const uint16_t* const* g
     a.head = head;
     a.nvec = (len - head) / 8;
   }
+  const void* k = rs_kernel_for(world, dtype);
+  const size_t smem = rs_smem_for_world(world);
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   void* args[] = {&a};
-  return cudaLaunchKernel(rs_kernel_for(world, dtype), dim3(grid), dim3(kRsThreads), args, 0, s);
+  return cudaLaunchKernel(k, dim3(grid), dim3(kRsTmaThreads), args, smem, s);
 }
 
 cudaError_t launch_finalize(void* ws, const int32_t* bucket_blocks, int64_t slots_full,
@@ -569,14 +800,24 @@ cudaError_t launch_finalize(void* ws, const int32_t* bucket_blocks, int64_t slot
 cudaError_t launch_update(int dtype, const float* R, float* master, float* m, float* v,
                           void* params, int64_t n, const void* ws, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
-  UpArgs a{R, master, m, v, params, n, (const WsHeader*)ws};
+  WsHeader* h = (WsHeader*)ws;
+  UpArgs a{R, master, m, v, params, n, h, &h->result.device_error};
   const void* k = dtype == ZERO_BF16 ? (const void*)adamw_cast_kernel<ZERO_BF16>
                                      : (const void*)adamw_cast_kernel<ZERO_FP16>;
-  int grid = 1;
-  cudaError_t e = persistent_grid(k, kUpThreads, (n + 7) / 8, &grid);
+  // the shared-memory opt-in is per function and device: set it before every launch
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kUpSmemBytes);
   if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kUpTmaThreads, kUpSmemBytes);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  int64_t grid = (int64_t)per_sm * sm_count();
+  const int64_t n_tiles = n / kUpTile;
+  if (grid > n_tiles) grid = n_tiles;
+  if (grid < 1) grid = 1;
   void* args[] = {&a};
-  return cudaLaunchKernel(k, dim3(grid), dim3(kUpThreads), args, 0, s);
+  return cudaLaunchKernel(k, dim3((unsigned)grid), dim3(kUpTmaThreads), args, kUpSmemBytes, s);
 }
 
 cudaError_t launch_cast(int dtype, const float* master, void* params, int64_t n,

@@ -101,10 +101,10 @@ extern "C" int zero_reduce_sumsq_noalloc(int32_t world_size, int32_t grad_dtype,
   int64_t blocks = (n + kNoallocBlockElems - 1) / kNoallocBlockElems;
   if (blocks < 1) blocks = 1;
   cudaStream_t s = (cudaStream_t)stream;
-  // the unchanged reduce-scatter kernel, one 8-element group per thread, its partial
-  // sums and block count written into the scratch array
-  e = launch_reduce_scatter(world_size, grad_dtype, g, reduced, 0, n, scratch,
-                            (int32_t*)(scratch + ZERO_NOALLOC_MAX_BLOCKS), (int)blocks, s);
+  // the reduce-scatter kernel with one block per 2048 elements, its partial sums and
+  // block count written into the scratch array
+  e = launch_reduce_scatter(world_size, grad_dtype, g, reduced, n, scratch,
+                            (int32_t*)(scratch + ZERO_NOALLOC_MAX_BLOCKS), nullptr, (int)blocks, s);
   if (e != cudaSuccess) return cuda_fail(e, "no-alloc reduce launch");
   noalloc_sum_kernel<<<1, kFinalizeThreads, 0, s>>>(scratch, (int32_t)blocks, sumsq);
   e = cudaGetLastError();

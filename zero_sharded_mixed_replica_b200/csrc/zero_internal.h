@@ -12,11 +12,11 @@
 
 namespace zero {
 
-// Reduce-scatter launch shape: 256 threads, 8 elements (one 16-byte half vector per
-// replica) per thread per group, at most kRsMaxBlocks blocks per bucket.
+// Reduce-scatter: partial-sum slots are reserved for one block per 256 groups of 8
+// elements, at most kRsMaxBlocks per bucket (a launch uses at most that many blocks).
 constexpr int kRsThreads = 256;
 constexpr int kRsMaxBlocks = 148 * 8;
-// Update launch shape.
+// Launch shape of the small grid-stride kernels (cast, replicate).
 constexpr int kUpThreads = 256;
 constexpr int kFinalizeThreads = 1024;
 
@@ -86,8 +86,8 @@ cudaError_t rs_grid(int64_t len, int world, int dtype, int* grid);
 // Launchers (kernels.cu). All return cudaSuccess or the launch error.
 cudaError_t launch_state_init(void* ws, const zero_scaler_cfg& cfg, cudaStream_t s);
 cudaError_t launch_reduce_scatter(int world, int dtype, const uint16_t* const* g, float* R,
-                                  int64_t start, int64_t len, double* partial,
-                                  int32_t* bucket_blocks, int grid, cudaStream_t s);
+                                  int64_t len, double* partial, int32_t* bucket_blocks,
+                                  int32_t* device_error, int grid, cudaStream_t s);
 cudaError_t launch_finalize(void* ws, const int32_t* bucket_blocks, int64_t slots_full,
                             const double* partial, int64_t n_buckets,
                             const zero_adamw_cfg& cfg, cudaStream_t s);
