@@ -53,6 +53,12 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--sweep", action="store_true",
+                    help="roofline sweep: 2^{24,26,28,30} x W in {1,2,4,8,16} x {bf16, fp16}; "
+                         "one JSON line per point")
+    ap.add_argument("--sweep-log2n", default="24,26,28,30")
+    ap.add_argument("--sweep-world", default="1,2,4,8,16")
+    ap.add_argument("--sweep-dtype", default="bf16,fp16")
     return ap.parse_args()
 
 
@@ -193,9 +199,9 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
     n_pad, W, nb = plan.n_pad, wl.world, plan.n_buckets
     sdev.init_master(wl, opt.master, sh)
     opt.cast_params()
-    # replica gradients: two slots of W bucket-sized buffers (or whole-model buffers
-    # when the model fits in one bucket)
-    L = min(wl.bucket, n_pad)
+    # replica gradients: streaming workloads use two slots of W bucket-sized buffers
+    # (indexed from the bucket start); resident ones whole-model buffers (flat index)
+    L = min(wl.bucket, n_pad) if wl.streaming else n_pad
     slots = [[torch.zeros(L, dtype=half, device=dev) for _ in range(W)] for _ in range(2)]
     scale = float(2.0 ** wl.init_scale_power) if wl.dynamic else 1.0
     for k in range(2):
@@ -251,6 +257,25 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
     clocks = sampler.stop()
     ms_total = start.elapsed_time(end)
     res = opt.result()
+
+    # Optional all-gather into per-rank copies (not part of the step: the gathered
+    # buffer is complete after the update). Timed apart on n_dst destinations that fit
+    # next to the resident state.
+    free_b, _ = torch.cuda.mem_get_info(dev)
+    n_dst = int(min(W, max(0, (free_b - (4 << 30)) // (2 * n_pad))))
+    k4 = None
+    if n_dst > 0:
+        dst = [torch.empty(n_pad, dtype=half, device=dev) for _ in range(n_dst)]
+        opt.all_gather(dst)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        opt.all_gather(dst)
+        e1.record(s)
+        torch.cuda.synchronize(dev)
+        k4_ms = e0.elapsed_time(e1)
+        k4 = {"n_dst": n_dst, "ms": k4_ms,
+              "gbs": (2 + 2 * n_dst) * n_pad / (k4_ms / 1e3) / 1e9}
+        del dst
 
     k1_ms = [a.elapsed_time(b) for a, b in ev_k1]
     k2_ms = [a.elapsed_time(b) for a, b in ev_k2]
@@ -310,6 +335,7 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
                          "finalize": sum(k2_ms) / len(k2_ms),
                          "adamw_cast": k3_avg},
             "reduce_scatter_gbs": k1_bytes / (k1_avg / 1e3) / 1e9,
+            "all_gather_copies": k4,
             "roofline": {
                 "kernel": "adamw_cast_kernel",
                 "bound": "hbm",
@@ -354,16 +380,16 @@ def run_e2e(args, wl, local_rank: int):
     W, nb = wl.world, plan.n_buckets
     sdev.init_master(wl, opt.master, s.cuda_stream)
     opt.cast_params()
-    L = min(wl.bucket, plan.n_pad)
+    L = min(wl.bucket, plan.n_pad) if wl.streaming else plan.n_pad
     half = {"bf16": torch.bfloat16, "fp16": torch.float16}[wl.gdtype]
-    # pinned host gradients: the same two-slot recipe as the device-resident run
-    host = [[torch.empty(L, dtype=torch.int16).pin_memory() for _ in range(W)] for _ in range(2)]
+    # pinned host gradients: the same recipe as the device-resident run
+    host = [[torch.zeros(L, dtype=torch.int16).pin_memory() for _ in range(W)] for _ in range(2)]
     for k in range(2):
         for r in range(W):
             synthgen.grads_host(0, min(L, wl.n), wl.seed, r, wl.slot(k + 1), wl.grad_sigma,
                                 wl.spike_frac, 1.0, wl.dtype_code,
                                 out=host[k][r].numpy().view(np.uint16))
-    staging = [torch.empty(L, dtype=half, device=dev) for _ in range(W)]
+    staging = [torch.empty(min(wl.bucket, plan.n_pad), dtype=half, device=dev) for _ in range(W)]
     h2d = 0
 
     def one(t):
@@ -393,6 +419,66 @@ def run_e2e(args, wl, local_rank: int):
     return out
 
 
+def run_sweep_point(wl, steps: int, local_rank: int) -> dict:
+    """All steps of one sweep point. Replica slots are regenerated before every step
+    (the loss scale in force for fp16, the +inf site at step 5) outside the timed part;
+    each step's kernels are timed with CUDA events on the launching stream."""
+    import torch
+
+    from synthgen import device as sdev
+    import zero_sharded_mixed_replica_b200 as zb
+
+    dev = torch.device("cuda", local_rank)
+    s = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(s)
+    sh = s.cuda_stream
+    half = {"bf16": torch.bfloat16, "fp16": torch.float16}[wl.gdtype]
+    scaler = zb.scaler_cfg(wl.dynamic, wl.init_scale_power, wl.loss_scale_window,
+                           wl.hysteresis, wl.min_loss_scale)
+    adamw = zb.adamw_cfg(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.max_grad_norm)
+    opt = zb.ZeroOptimizer([t.shape for t in wl.tensors], wl.world, wl.bucket, wl.gdtype,
+                           wl.align, scaler, adamw, device=str(dev), stream=s)
+    plan = opt.plan
+    sdev.init_master(wl, opt.master, sh)
+    opt.cast_params()
+    L = min(wl.bucket, plan.n_pad)
+    slots = [[torch.empty(L, dtype=half, device=dev) for _ in range(wl.world)] for _ in range(2)]
+    scale = float(2.0 ** wl.init_scale_power) if wl.dynamic else 1.0
+    applied, skipped = [], []
+    for t in range(1, steps + 1):
+        bufs = slots[(t - 1) % 2]
+        sdev.fill_grads(wl, bufs, 0, L, t, scale, sh)
+        sdev.plant_infs(wl, bufs, t, wl.bucket)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        for bk in range(plan.n_buckets):
+            opt.reduce_scatter_bucket(bk, bufs, base_offset=bk * wl.bucket)
+        opt.step()
+        b.record(s)
+        res = opt.result()
+        (skipped if res["skipped"] else applied).append(a.elapsed_time(b))
+        scale = float(res["next_scale"]) if wl.dynamic else 1.0
+    ms = statistics.median(applied[1:] if len(applied) > 2 else applied)
+    W = wl.world
+    out = {
+        "point": wl.name, "params": plan.n, "W": W, "grad_dtype": wl.gdtype,
+        "buckets": plan.n_buckets, "steps": steps,
+        "ms_per_applied_step_median": ms,
+        "params_per_s": plan.n / (ms / 1e3),
+        "hbm_gbs_schedule": schedule_bytes_per_param(W) * plan.n_pad / (ms / 1e3) / 1e9,
+        "hbm_gbs_model": model_bytes_per_param(W) * plan.n / (ms / 1e3) / 1e9,
+        "first_step_ms": (applied + skipped)[0],
+        "skipped_steps": len(skipped),
+        "ms_skipped_step_median": statistics.median(skipped) if skipped else None,
+    }
+    peak, kind = measured_peaks()
+    out["frac_of_8tbs_schedule"] = out["hbm_gbs_schedule"] / 8000.0
+    out["frac_of_peak_schedule"] = out["hbm_gbs_schedule"] / peak
+    del opt, slots
+    torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------------------- oracle arm
 
 def oracle_sample_run(wl, seconds: float, max_steps: int = 0, warmup: int = 0):
@@ -416,18 +502,26 @@ def oracle_sample_run(wl, seconds: float, max_steps: int = 0, warmup: int = 0):
     params = oracle.f32_to_half(master, dt)
     cfg, hp = oracle.workload_cfg(wl)
     st = oracle.state_init(cfg)
-    for _ in range(warmup):
-        oracle.step(grads, dt, wl.bucket, R, master, m, v, params, dt, cfg, hp, st)
-    steps = 0
-    t0 = time.perf_counter()
-    while True:
-        oracle.step(grads, dt, wl.bucket, R, master, m, v, params, dt, cfg, hp, st)
-        steps += 1
-        el = time.perf_counter() - t0
-        if (max_steps and steps >= max_steps) or (not max_steps and el >= seconds):
-            break
+    # the oracle is single-threaded: pin the timed part to one host core
+    prev_affinity = os.sched_getaffinity(0)
+    core = min(prev_affinity)
+    os.sched_setaffinity(0, {core})
+    try:
+        for _ in range(warmup):
+            oracle.step(grads, dt, wl.bucket, R, master, m, v, params, dt, cfg, hp, st)
+        steps = 0
+        t0 = time.perf_counter()
+        while True:
+            oracle.step(grads, dt, wl.bucket, R, master, m, v, params, dt, cfg, hp, st)
+            steps += 1
+            el = time.perf_counter() - t0
+            if (max_steps and steps >= max_steps) or (not max_steps and el >= seconds):
+                break
+    finally:
+        os.sched_setaffinity(0, prev_affinity)
     desc = (f"{n} params ({wl.name} flat indices 0..{n - 1}), W={wl.world} {wl.gdtype} replicas, "
-            f"{steps} full oracle steps (reduce, sum of squares, finalize, AdamW + cast)")
+            f"{steps} full oracle steps (reduce, sum of squares, finalize, AdamW + cast), "
+            f"pinned to host core {core}; params/s of the sample, not extrapolated")
     return n * steps / el, desc, steps, el
 
 
@@ -469,6 +563,15 @@ def main():
         out = run_reference(args, rank)
         if out is not None:
             print(json.dumps(out), flush=True)
+        return
+
+    if args.sweep:
+        import synthgen
+        for log2n in [int(x) for x in args.sweep_log2n.split(",")]:
+            for W in [int(x) for x in args.sweep_world.split(",")]:
+                for dt in args.sweep_dtype.split(","):
+                    wl = synthgen.sweep(log2n, W, dt)
+                    print(json.dumps(run_sweep_point(wl, wl.steps, local_rank)), flush=True)
         return
 
     import torch

@@ -258,6 +258,49 @@ ZERO_API int zero_all_gather(const zero_plan* plan, const void* params, void* co
  * ZERO_EDEVICE (with *out filled) if a kernel reported a timed-out internal wait. */
 ZERO_API int zero_get_result(const void* workspace, zero_step_result* out, void* stream);
 
+/* ---------------------------------------------------------------- one rank of W processes
+ * A real data-parallel run: W processes, one GPU each, the same plan on every rank;
+ * rank r owns partition r ([Z1] 2.1: each GPU updates only its own partition; [Z3]: each
+ * GPU keeps only the gradient slice for its own parameters) and holds its fp32 master,
+ * m, v and reduced gradient for that partition only (p elements each). One step on rank r:
+ *   for every bucket b that meets partition r (in order):
+ *       zero_reduce_scatter_segment(b, r): reduced_local = rank-ordered fp32 sum of the W
+ *       replicas over bucket b ∩ partition r. replica_grads[q] is rank q's gradient
+ *       buffer mapped into this process (CUDA IPC, NVLink peer reads; no multicast);
+ *       the caller orders it after every rank finished writing bucket b.
+ *   zero_step_local_sumsq(r): this rank's fp64 sum of squares into *sumsq_out (device).
+ *   exchange: the caller gathers the W sums into sumsq_ranks (device, rank order), e.g.
+ *       with an all-gather.
+ *   zero_step_finalize_ranks: S = ((s_0 + s_1) + ...) + s_{W-1}, then the same scalar
+ *       step as zero_step_finalize -- identical on every rank.
+ *   zero_step_update_partition(r): AdamW on the local arrays; the half result goes to
+ *       params_dst[d] + r*p for every d -- this rank's own gathered buffer and, mapped
+ *       over CUDA IPC, its peers' (the all-gather fused into the update as P2P stores),
+ *       or only its own when the caller all-gathers afterwards.
+ * Errors as above; ESTATE when a segment is reduced twice, a bucket outside the rank's
+ * partition is reduced, or the calls come out of order. */
+ZERO_API int zero_reduce_scatter_segment(zero_plan* plan, int64_t bucket, int32_t rank,
+                                         int32_t grad_dtype, const void* const* replica_grads,
+                                         int64_t replica_base_offset, float* reduced_local,
+                                         void* workspace, void* stream);
+ZERO_API int zero_step_local_sumsq(zero_plan* plan, int32_t rank, void* workspace,
+                                   double* sumsq_out, void* stream);
+ZERO_API int zero_step_finalize_ranks(zero_plan* plan, const zero_adamw_cfg* cfg,
+                                      const double* sumsq_ranks, void* workspace, void* stream);
+ZERO_API int zero_step_update_partition(zero_plan* plan, int32_t rank, float* master_local,
+                                        float* exp_avg_local, float* exp_avg_sq_local,
+                                        const float* reduced_local, void* const* params_dst,
+                                        int32_t n_dst, int32_t param_dtype,
+                                        const void* workspace, void* stream);
+
+/* Peer memory: CUDA IPC handles (ZERO_IPC_HANDLE_BYTES opaque bytes) so that rank q's
+ * buffers can be read and written by the other ranks' kernels over NVLink. The caller
+ * moves the handle bytes between processes (e.g. an all-gather of objects). */
+ZERO_API int zero_ipc_handle_bytes(void);
+ZERO_API int zero_ipc_get_handle(const void* device_ptr, void* handle_out);
+ZERO_API int zero_ipc_open_handle(const void* handle, void** device_ptr);
+ZERO_API int zero_ipc_close(void* device_ptr);
+
 /* ---------------------------------------------------------------- no-alloc variant
  * zero_reduce_sumsq_noalloc has no counterpart in the pages. It is for callers that
  * cannot allocate device memory for a workspace: for example a C plugin that its host

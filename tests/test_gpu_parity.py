@@ -360,3 +360,44 @@ def test_guard_regions_untouched():
     for t in big.values():
         assert torch.all(t[n:] == 7.0)
     assert torch.all(pbig[n:] == 3.0)
+
+
+# ----------------------------------------------------------------------------- sweep
+
+def _check_streaming(wl, idx=None, steps=None):
+    scalars = oracle.streaming_scalars(wl, steps=steps)
+    opt, results = run_streaming(wl, steps=steps)
+    for res, sc in zip(results, scalars):
+        check_scalars(res, sc.as_dict())
+    if idx is None:
+        idx = np.arange(opt.plan.n_pad, dtype=np.int64)
+    want = oracle.streaming_samples(wl, idx, scalars)
+    it = torch.from_numpy(idx).cuda()
+    assert np.array_equal(opt.reduced[it].cpu().numpy().view(np.uint32), want["R"].view(np.uint32))
+    for name, t in (("master", opt.master), ("m", opt.exp_avg), ("v", opt.exp_avg_sq)):
+        check_state(name, t[it].cpu().numpy(), want[name], 1)
+    assert half_ulp_distance(to_np(opt.params[it]), want["params"]).max() <= 1
+    return results
+
+
+@pytest.mark.parametrize("world,dtype", [(1, "bf16"), (16, "bf16"), (1, "fp16"), (16, "fp16")])
+def test_sweep_2_24_every_element(world, dtype):
+    """Sweep point 2^24 x W x dtype, 10 steps (fp16: dynamic scaler with one +inf at
+    step 5), every element compared."""
+    wl = synthgen.sweep(24, world, dtype)
+    results = _check_streaming(wl)
+    if dtype == "fp16":
+        assert [r["skipped"] for r in results] == [0, 0, 0, 0, 1, 0, 0, 0, 0, 0]
+        assert results[-1]["adam_t"] == 9
+
+
+def test_sweep_2_30_w16_sampled():
+    """The largest sweep point (2^30 params, W=16, 6 buckets of 2e8), 3 steps,
+    scalars from the full gradient stream and ~4k sampled elements."""
+    wl = synthgen.sweep(30, 16, "bf16", steps=3)
+    rng = np.random.default_rng(5)
+    n = wl.n
+    idx = np.unique(np.concatenate([rng.integers(0, n, 4096), [0, n - 1],
+                                    [b * wl.bucket + d for b in range(1, 6) for d in (-1, 0)],
+                                    [r * (n // 16) + d for r in range(1, 16) for d in (-1, 0)]]))
+    _check_streaming(wl, idx.astype(np.int64))

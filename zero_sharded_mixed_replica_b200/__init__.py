@@ -119,6 +119,15 @@ def _load():
         "zero_step_update": [vp, vp, vp, vp, vp, vp, i32, vp, vp],
         "zero_all_gather": [vp, vp, vp, i32, i32, vp],
         "zero_get_result": [vp, P(StepResult), vp],
+        "zero_reduce_scatter_segment": [vp, i64, i32, i32, vp, i64, vp, vp, vp],
+        "zero_step_local_sumsq": [vp, i32, vp, vp, vp],
+        "zero_step_finalize_ranks": [vp, P(AdamWCfg), vp, vp, vp],
+        "zero_step_update_partition": [vp, i32, vp, vp, vp, vp, vp, i32, i32, vp, vp],
+        "zero_ipc_handle_bytes": [],
+        "zero_ipc_get_handle": [vp, vp],
+        "zero_ipc_open_handle": [vp, P(vp)],
+        "zero_ipc_close": [vp],
+        "zero_reduce_sumsq_noalloc": [i32, i32, vp, i64, vp, vp, vp],
         "zero_last_error": [],
         "zero_abi_version": [],
     }
@@ -321,6 +330,60 @@ def zero_get_result(workspace, stream=None) -> dict:
 
 def zero_abi_version() -> int:
     return lib.zero_abi_version()
+
+
+# ---------------------------------------------------------------------------- one rank of W
+
+def zero_reduce_scatter_segment(plan: Plan, bucket: int, rank: int, grad_dtype,
+                                replica_grads: Sequence, replica_base_offset: int,
+                                reduced_local, workspace, stream=None) -> None:
+    _check(lib.zero_reduce_scatter_segment(plan.handle, bucket, rank, _dtype(grad_dtype),
+                                           _ptr_array(replica_grads), int(replica_base_offset),
+                                           _addr(reduced_local), _addr(workspace),
+                                           _stream(stream)))
+
+
+def zero_step_local_sumsq(plan: Plan, rank: int, workspace, sumsq_out, stream=None) -> None:
+    _check(lib.zero_step_local_sumsq(plan.handle, rank, _addr(workspace), _addr(sumsq_out),
+                                     _stream(stream)))
+
+
+def zero_step_finalize_ranks(plan: Plan, cfg: AdamWCfg, sumsq_ranks, workspace,
+                             stream=None) -> None:
+    _check(lib.zero_step_finalize_ranks(plan.handle, ctypes.byref(cfg), _addr(sumsq_ranks),
+                                        _addr(workspace), _stream(stream)))
+
+
+def zero_step_update_partition(plan: Plan, rank: int, master_local, exp_avg_local,
+                               exp_avg_sq_local, reduced_local, params_dst: Sequence,
+                               param_dtype, workspace, stream=None) -> None:
+    _check(lib.zero_step_update_partition(
+        plan.handle, rank, _addr(master_local), _addr(exp_avg_local), _addr(exp_avg_sq_local),
+        _addr(reduced_local), _ptr_array(params_dst), len(params_dst), _dtype(param_dtype),
+        _addr(workspace), _stream(stream)))
+
+
+def zero_ipc_get_handle(device_ptr) -> bytes:
+    buf = ctypes.create_string_buffer(lib.zero_ipc_handle_bytes())
+    _check(lib.zero_ipc_get_handle(_addr(device_ptr), buf))
+    return buf.raw
+
+
+def zero_ipc_open_handle(handle: bytes) -> int:
+    p = ctypes.c_void_p()
+    _check(lib.zero_ipc_open_handle(ctypes.create_string_buffer(handle, len(handle)),
+                                    ctypes.byref(p)))
+    return int(p.value)
+
+
+def zero_ipc_close(device_ptr: int) -> None:
+    _check(lib.zero_ipc_close(device_ptr))
+
+
+def zero_reduce_sumsq_noalloc(world_size: int, grad_dtype, replica_grads: Sequence, n: int,
+                              reduced, sumsq, stream=None) -> None:
+    _check(lib.zero_reduce_sumsq_noalloc(world_size, _dtype(grad_dtype), _ptr_array(replica_grads),
+                                         int(n), _addr(reduced), _addr(sumsq), _stream(stream)))
 
 
 from .optimizer import ZeroOptimizer  # noqa: E402  (torch plumbing around the calls above)

@@ -407,7 +407,8 @@ int zero_step_update(zero_plan* plan, float* master, float* exp_avg, float* exp_
     return fail(ZERO_EALIGN, "step buffers must be 16-byte aligned");
   if (!plan->finalized)
     return fail(ZERO_ESTATE, "zero_step_update without a zero_step_finalize before it");
-  cudaError_t e = launch_update(param_dtype, reduced, master, exp_avg, exp_avg_sq, params,
+  void* dst[1] = {params};
+  cudaError_t e = launch_update(param_dtype, reduced, master, exp_avg, exp_avg_sq, dst, 1,
                                 plan->n_pad, workspace, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "update launch");
   plan->finalized = false;
@@ -459,6 +460,159 @@ int zero_get_result(const void* workspace, zero_step_result* out, void* stream) 
   if (out->device_error)
     return fail(ZERO_EDEVICE, "a kernel gave up on a bounded internal wait (code " +
                                   std::to_string(out->device_error) + "); outputs are incomplete");
+  return ZERO_OK;
+}
+
+// ------------------------------------------------------------------ one rank of W processes
+
+namespace {
+// buckets [b0, b1) that meet partition `rank`
+void rank_buckets(const zero_plan* plan, int32_t rank, int64_t* b0, int64_t* b1) {
+  if (plan->p == 0 || plan->n_buckets == 0) {
+    *b0 = *b1 = 0;
+    return;
+  }
+  const int64_t lo = (int64_t)rank * plan->p, hi = lo + plan->p;
+  *b0 = lo / plan->bucket;
+  *b1 = (hi - 1) / plan->bucket + 1;
+}
+}  // namespace
+
+int zero_reduce_scatter_segment(zero_plan* plan, int64_t bucket, int32_t rank,
+                                int32_t grad_dtype, const void* const* replica_grads,
+                                int64_t replica_base_offset, float* reduced_local,
+                                void* workspace, void* stream) {
+  if (!plan) return fail(ZERO_EINVAL, "plan is NULL");
+  if (rank < 0 || rank >= plan->world) return fail(ZERO_EINVAL, "rank out of range");
+  if (int rc = check_bucket_call(plan, bucket, grad_dtype, reduced_local, workspace)) return rc;
+  if (!replica_grads) return fail(ZERO_EINVAL, "replica_grads is NULL");
+  int64_t b0, b1;
+  rank_buckets(plan, rank, &b0, &b1);
+  if (bucket < b0 || bucket >= b1)
+    return fail(ZERO_EINVAL, "bucket " + std::to_string(bucket) + " does not meet partition " +
+                                 std::to_string(rank));
+  const int64_t bs = bucket * plan->bucket, be = bs + bucket_len(plan, bucket);
+  const int64_t ps = (int64_t)rank * plan->p, pe = ps + plan->p;
+  const int64_t lo = bs > ps ? bs : ps, hi = be < pe ? be : pe;
+  if (replica_base_offset < 0 || replica_base_offset > lo)
+    return fail(ZERO_EINVAL, "replica_base_offset must be in [0, segment start]");
+  const uint16_t* g[ZERO_MAX_WORLD];
+  for (int r = 0; r < plan->world; ++r) {
+    if (!replica_grads[r]) return fail(ZERO_EINVAL, "replica_grads[" + std::to_string(r) + "] is NULL");
+    if (!aligned16(replica_grads[r]))
+      return fail(ZERO_EALIGN, "replica_grads[" + std::to_string(r) + "] is not 16-byte aligned");
+    g[r] = (const uint16_t*)replica_grads[r] + (lo - replica_base_offset);
+  }
+  const int64_t len = hi - lo;
+  int grid = 1;
+  cudaError_t e = rs_grid(len, plan->world, grad_dtype, &grid);
+  if (e != cudaSuccess) return cuda_fail(e, "reduce-scatter occupancy query");
+  e = launch_reduce_scatter(plan->world, grad_dtype, g, reduced_local + (lo - ps), len,
+                            ws_partial(plan, workspace) + bucket * plan->slots_full,
+                            ws_bucket_blocks(plan, workspace) + bucket,
+                            &((WsHeader*)workspace)->result.device_error, grid,
+                            (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "reduce-scatter launch");
+  plan->reduced[bucket] = 1;
+  plan->reduced_count += 1;
+  return ZERO_OK;
+}
+
+int zero_step_local_sumsq(zero_plan* plan, int32_t rank, void* workspace, double* sumsq_out,
+                          void* stream) {
+  if (!plan || !workspace || !sumsq_out) return fail(ZERO_EINVAL, "NULL argument");
+  if (rank < 0 || rank >= plan->world) return fail(ZERO_EINVAL, "rank out of range");
+  if (((uintptr_t)sumsq_out & 7u) != 0) return fail(ZERO_EALIGN, "sumsq_out must be 8-byte aligned");
+  int64_t b0, b1;
+  rank_buckets(plan, rank, &b0, &b1);
+  for (int64_t b = b0; b < b1; ++b)
+    if (!plan->reduced[b])
+      return fail(ZERO_ESTATE, "segment of bucket " + std::to_string(b) + " not reduced yet");
+  if (plan->reduced_count != b1 - b0)
+    return fail(ZERO_ESTATE, "buckets outside this rank's partition were reduced");
+  cudaError_t e = launch_local_sumsq(ws_bucket_blocks(plan, workspace), plan->slots_full,
+                                     ws_partial(plan, workspace), b0, b1, sumsq_out,
+                                     (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "local sum launch");
+  plan->local_summed = true;
+  return ZERO_OK;
+}
+
+int zero_step_finalize_ranks(zero_plan* plan, const zero_adamw_cfg* cfg,
+                             const double* sumsq_ranks, void* workspace, void* stream) {
+  if (!plan || !workspace || !sumsq_ranks) return fail(ZERO_EINVAL, "NULL argument");
+  if (int rc = check_adamw(cfg)) return rc;
+  if (!plan->local_summed)
+    return fail(ZERO_ESTATE, "zero_step_finalize_ranks before zero_step_local_sumsq");
+  cudaError_t e = launch_finalize_ranks(workspace, sumsq_ranks, plan->world, *cfg,
+                                        (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "finalize launch");
+  plan->reduced.assign((size_t)plan->n_buckets, 0);
+  plan->reduced_count = 0;
+  plan->local_summed = false;
+  plan->finalized = true;
+  return ZERO_OK;
+}
+
+int zero_step_update_partition(zero_plan* plan, int32_t rank, float* master_local,
+                               float* exp_avg_local, float* exp_avg_sq_local,
+                               const float* reduced_local, void* const* params_dst,
+                               int32_t n_dst, int32_t param_dtype, const void* workspace,
+                               void* stream) {
+  if (!plan || !workspace || !params_dst) return fail(ZERO_EINVAL, "NULL argument");
+  if (rank < 0 || rank >= plan->world) return fail(ZERO_EINVAL, "rank out of range");
+  if (n_dst < 1 || n_dst > ZERO_MAX_WORLD)
+    return fail(ZERO_EINVAL, "n_dst must be in [1, " + std::to_string(ZERO_MAX_WORLD) + "]");
+  if (int rc = check_dtype(param_dtype, "zero_step_update_partition")) return rc;
+  if (plan->p > 0 && (!master_local || !exp_avg_local || !exp_avg_sq_local || !reduced_local))
+    return fail(ZERO_EINVAL, "NULL argument");
+  if (!aligned16(master_local) || !aligned16(exp_avg_local) || !aligned16(exp_avg_sq_local) ||
+      !aligned16(reduced_local) || !aligned16(workspace))
+    return fail(ZERO_EALIGN, "partition buffers must be 16-byte aligned");
+  void* dst[ZERO_MAX_WORLD];
+  for (int d = 0; d < n_dst; ++d) {
+    if (!params_dst[d] && plan->p > 0) return fail(ZERO_EINVAL, "params_dst has a NULL entry");
+    // this rank's slice of each gathered buffer
+    dst[d] = (uint16_t*)params_dst[d] + (int64_t)rank * plan->p;
+    if (!aligned16(dst[d]))
+      return fail(ZERO_EALIGN, "params_dst[" + std::to_string(d) + "] + rank*p is not 16-byte aligned");
+  }
+  if (!plan->finalized)
+    return fail(ZERO_ESTATE, "zero_step_update_partition without a finalize before it");
+  cudaError_t e = launch_update(param_dtype, reduced_local, master_local, exp_avg_local,
+                                exp_avg_sq_local, dst, n_dst, plan->p, workspace,
+                                (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "update launch");
+  plan->finalized = false;
+  return ZERO_OK;
+}
+
+// ------------------------------------------------------------------ peer memory
+
+int zero_ipc_handle_bytes(void) { return (int)sizeof(cudaIpcMemHandle_t); }
+
+int zero_ipc_get_handle(const void* device_ptr, void* handle_out) {
+  if (!device_ptr || !handle_out) return fail(ZERO_EINVAL, "NULL argument");
+  cudaIpcMemHandle_t h;
+  cudaError_t e = cudaIpcGetMemHandle(&h, (void*)device_ptr);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaIpcGetMemHandle");
+  memcpy(handle_out, &h, sizeof h);
+  return ZERO_OK;
+}
+
+int zero_ipc_open_handle(const void* handle, void** device_ptr) {
+  if (!handle || !device_ptr) return fail(ZERO_EINVAL, "NULL argument");
+  cudaIpcMemHandle_t h;
+  memcpy(&h, handle, sizeof h);
+  cudaError_t e = cudaIpcOpenMemHandle(device_ptr, h, cudaIpcMemLazyEnablePeerAccess);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaIpcOpenMemHandle");
+  return ZERO_OK;
+}
+
+int zero_ipc_close(void* device_ptr) {
+  if (!device_ptr) return fail(ZERO_EINVAL, "NULL argument");
+  cudaError_t e = cudaIpcCloseMemHandle(device_ptr);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaIpcCloseMemHandle");
   return ZERO_OK;
 }
 

@@ -394,20 +394,10 @@ __device__ double pow_int(double x, int64_t n) {
   return result;
 }
 
-__global__ void __launch_bounds__(kFinalizeThreads)
-    finalize_kernel(WsHeader* h, const int32_t* __restrict__ bucket_blocks, int64_t slots_full,
-                    const double* __restrict__ partial, int64_t n_buckets, zero_adamw_cfg cfg) {
-  // S: fixed order -- each thread walks buckets in order and its own slots in order,
-  // then the block tree.
-  double acc = 0.0;
-  for (int64_t b = 0; b < n_buckets; ++b) {
-    const int32_t nb = bucket_blocks[b];
-    const double* p = partial + b * slots_full;
-    for (int j = threadIdx.x; j < nb; j += kFinalizeThreads) acc = __dadd_rn(acc, p[j]);
-  }
-  const double S = block_sum<kFinalizeThreads>(acc);
-  if (threadIdx.x != 0) return;
-
+// Everything the step decides from S, done by one thread: overflow (S not finite), the
+// unscaled norm, the clip coefficient, the one fp32 multiplier k, the loss-scaler
+// transition, the step counter and the fp32 constants of the update.
+__device__ void finalize_scalars(WsHeader* h, double S, const zero_adamw_cfg& cfg) {
   const float scale = h->scale;
   const int32_t overflow = isfinite(S) ? 0 : 1;
   const double norm = __ddiv_rn(__dsqrt_rn(S), (double)scale);
@@ -463,6 +453,45 @@ __global__ void __launch_bounds__(kFinalizeThreads)
   r.adam_t = t;  // r.device_error is left as it is: sticky until zero_state_init
 }
 
+// Sum of the partial-sum slots of buckets [b0, b1) in a fixed order: each thread walks
+// the buckets in order and its own slots in order, then the block tree. Valid in thread 0.
+__device__ double sum_bucket_slots(const int32_t* __restrict__ bucket_blocks, int64_t slots_full,
+                                   const double* __restrict__ partial, int64_t b0, int64_t b1) {
+  double acc = 0.0;
+  for (int64_t b = b0; b < b1; ++b) {
+    const int32_t nb = bucket_blocks[b];
+    const double* p = partial + b * slots_full;
+    for (int j = threadIdx.x; j < nb; j += kFinalizeThreads) acc = __dadd_rn(acc, p[j]);
+  }
+  return block_sum<kFinalizeThreads>(acc);
+}
+
+// Single process: S over every bucket, then the scalar step.
+__global__ void __launch_bounds__(kFinalizeThreads)
+    finalize_kernel(WsHeader* h, const int32_t* __restrict__ bucket_blocks, int64_t slots_full,
+                    const double* __restrict__ partial, int64_t n_buckets, zero_adamw_cfg cfg) {
+  const double S = sum_bucket_slots(bucket_blocks, slots_full, partial, 0, n_buckets);
+  if (threadIdx.x == 0) finalize_scalars(h, S, cfg);
+}
+
+// One rank: the sum over the buckets its partition meets, for the cross-rank exchange.
+__global__ void __launch_bounds__(kFinalizeThreads)
+    local_sumsq_kernel(const int32_t* __restrict__ bucket_blocks, int64_t slots_full,
+                       const double* __restrict__ partial, int64_t b0, int64_t b1,
+                       double* out) {
+  const double S = sum_bucket_slots(bucket_blocks, slots_full, partial, b0, b1);
+  if (threadIdx.x == 0) *out = S;
+}
+
+// One rank, after the exchange: S = ((s_0 + s_1) + ...) + s_{W-1} in rank order, so every
+// rank computes the same S, then the scalar step.
+__global__ void finalize_ranks_kernel(WsHeader* h, const double* __restrict__ s_ranks,
+                                      int32_t world, zero_adamw_cfg cfg) {
+  double S = s_ranks[0];
+  for (int32_t r = 1; r < world; ++r) S = __dadd_rn(S, s_ranks[r]);
+  finalize_scalars(h, S, cfg);
+}
+
 // ================================================================== K3: AdamW + cast
 
 struct UpArgs {
@@ -470,7 +499,8 @@ struct UpArgs {
   float* p;
   float* m;
   float* v;
-  void* out;  // gathered half buffer
+  uint16_t* out[ZERO_MAX_WORLD];  // gathered half buffers (element 0 of this range)
+  int32_t n_out;
   int64_t n;
   const WsHeader* h;
   int32_t* device_error;  // &h->result.device_error
@@ -539,7 +569,6 @@ __global__ void __launch_bounds__(kUpTmaThreads, 1)
 
   const int64_t n_tiles = a.n / kUpTile;
   const int64_t G = gridDim.x;
-  uint16_t* out = (uint16_t*)a.out;
 
   if (tid >= kUpConsumers) {
     // producer warp: one thread issues the bulk copies
@@ -593,7 +622,8 @@ __global__ void __launch_bounds__(kUpTmaThreads, 1)
       st_f4(a.p + off + e, p.x, p.y, p.z, p.w);
       st_f4(a.m + off + e, m.x, m.y, m.z, m.w);
       st_f4(a.v + off + e, v.x, v.y, v.z, v.w);
-      *(uint2*)(out + off + e) = make_uint2(pack2<DT>(p.x, p.y), pack2<DT>(p.z, p.w));
+      const uint2 hv = make_uint2(pack2<DT>(p.x, p.y), pack2<DT>(p.z, p.w));
+      for (int d = 0; d < a.n_out; ++d) *(uint2*)(a.out[d] + off + e) = hv;
     }
     __syncwarp();
     if ((tid & 31) == 0) mbar_arrive(&empty[st]);
@@ -607,7 +637,8 @@ __global__ void __launch_bounds__(kUpTmaThreads, 1)
       a.p[i] = p;
       a.m[i] = m;
       a.v[i] = v;
-      out[i] = (uint16_t)float_to_half_bits<DT>(p);
+      const uint16_t hb = (uint16_t)float_to_half_bits<DT>(p);
+      for (int d = 0; d < a.n_out; ++d) a.out[d][i] = hb;
     }
   }
 }
@@ -797,11 +828,35 @@ cudaError_t launch_finalize(void* ws, const int32_t* bucket_blocks, int64_t slot
   return cudaGetLastError();
 }
 
+cudaError_t launch_local_sumsq(const int32_t* bucket_blocks, int64_t slots_full,
+                               const double* partial, int64_t b0, int64_t b1, double* out,
+                               cudaStream_t s) {
+  local_sumsq_kernel<<<1, kFinalizeThreads, 0, s>>>(bucket_blocks, slots_full, partial, b0, b1,
+                                                    out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize_ranks(void* ws, const double* s_ranks, int world,
+                                  const zero_adamw_cfg& cfg, cudaStream_t s) {
+  finalize_ranks_kernel<<<1, 1, 0, s>>>((WsHeader*)ws, s_ranks, world, cfg);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_update(int dtype, const float* R, float* master, float* m, float* v,
-                          void* params, int64_t n, const void* ws, cudaStream_t s) {
+                          void* const* params, int n_params, int64_t n, const void* ws,
+                          cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   WsHeader* h = (WsHeader*)ws;
-  UpArgs a{R, master, m, v, params, n, h, &h->result.device_error};
+  UpArgs a;
+  a.R = R;
+  a.p = master;
+  a.m = m;
+  a.v = v;
+  for (int d = 0; d < ZERO_MAX_WORLD; ++d) a.out[d] = d < n_params ? (uint16_t*)params[d] : nullptr;
+  a.n_out = n_params;
+  a.n = n;
+  a.h = h;
+  a.device_error = &h->result.device_error;
   const void* k = dtype == ZERO_BF16 ? (const void*)adamw_cast_kernel<ZERO_BF16>
                                      : (const void*)adamw_cast_kernel<ZERO_FP16>;
   // the shared-memory opt-in is per function and device: set it before every launch

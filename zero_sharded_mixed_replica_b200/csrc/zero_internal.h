@@ -67,6 +67,7 @@ struct zero_plan {
   std::vector<uint8_t> reduced;
   int64_t reduced_count = 0;
   bool finalized = false;  // finalize ran and no update consumed it yet
+  bool local_summed = false;  // one rank: its local sum of squares was taken this step
   size_t ws_bucket_blocks_off = 0;  // int32 per bucket: blocks of its last launch
   size_t ws_partial_off = 0;        // double per slot
   size_t ws_bytes = 0;
@@ -92,7 +93,13 @@ cudaError_t launch_finalize(void* ws, const int32_t* bucket_blocks, int64_t slot
                             const double* partial, int64_t n_buckets,
                             const zero_adamw_cfg& cfg, cudaStream_t s);
 cudaError_t launch_update(int dtype, const float* R, float* master, float* m, float* v,
-                          void* params, int64_t n, const void* ws, cudaStream_t s);
+                          void* const* params, int n_params, int64_t n, const void* ws,
+                          cudaStream_t s);
+cudaError_t launch_local_sumsq(const int32_t* bucket_blocks, int64_t slots_full,
+                               const double* partial, int64_t b0, int64_t b1, double* out,
+                               cudaStream_t s);
+cudaError_t launch_finalize_ranks(void* ws, const double* s_ranks, int world,
+                                  const zero_adamw_cfg& cfg, cudaStream_t s);
 cudaError_t launch_cast(int dtype, const float* master, void* params, int64_t n,
                         cudaStream_t s);
 cudaError_t launch_replicate(const void* src, void* const* dst, int n_dst, int64_t n_halves,

@@ -1,0 +1,159 @@
+"""The ZeRO step across W processes, one GPU each (rank r owns partition r).
+
+The orders of work and exchange live in `DistributedZeroStep`; what runs on a device
+lives in a backend. `CudaRankBackend` is the product backend: peers' gradient and
+gathered-parameter buffers are mapped into each process with CUDA IPC, the
+reduce-scatter reads them over NVLink inside the bucket kernel (rank-ordered fp32 sum,
+as on one GPU), and the update writes this rank's half values into every rank's
+gathered buffer (the all-gather fused into the update) -- or, with
+`fused_all_gather=False`, into its own buffer followed by a collective all-gather.
+The only collectives are one all-gather of the W fp64 sums of squares (rank order, so
+every rank computes the same norm, clip and loss-scale decision) and the stream-ordered
+barriers that separate writers from peer readers.
+
+Sources: [Z1] "ZeRO技术解析" 2.1 (parameters split into N parts, gradients
+reduce-scattered, each GPU updates its own partition, parameters gathered with
+all-gather) and 2.2 (bucketed communication); [Z3] "ZeRO 和分片优化器" technical
+insight (each GPU keeps only its own gradient slice).
+"""
+from __future__ import annotations
+
+from typing import List, Optional, Sequence
+
+import torch
+import torch.distributed as dist
+
+from . import (AdamWCfg, Plan, ScalerCfg, adamw_cfg, scaler_cfg, zero_get_result,
+               zero_ipc_close, zero_ipc_get_handle, zero_ipc_open_handle,
+               zero_reduce_scatter_segment, zero_state_init, zero_step_finalize_ranks,
+               zero_step_local_sumsq, zero_step_update_partition)
+
+_TORCH_HALF = {"bf16": torch.bfloat16, "fp16": torch.float16}
+
+
+def partition_buckets(plan_n_pad: int, world: int, bucket: int, rank: int) -> range:
+    """Buckets that meet partition `rank` (each such bucket holds exactly one of the
+    rank's work segments)."""
+    p = plan_n_pad // world
+    if p == 0:
+        return range(0)
+    lo, hi = rank * p, (rank + 1) * p
+    return range(lo // bucket, (hi - 1) // bucket + 1)
+
+
+class DistributedZeroStep:
+    """One optimizer step on this rank. `backend` does the device work; `group` is the
+    process group of the W ranks (NCCL for CUDA tensors, gloo for CPU tensors)."""
+
+    def __init__(self, backend, group=None):
+        self.backend = backend
+        self.group = group
+        self.rank = backend.rank
+        self.world = backend.world
+        self.buckets = partition_buckets(backend.n_pad, self.world, backend.bucket, self.rank)
+
+    def step(self):
+        be = self.backend
+        # every rank has finished writing this step's gradients before any peer reads them
+        be.before_peer_reads(self.group)
+        for b in self.buckets:
+            be.reduce_segment(b)
+        s_local = be.local_sumsq()
+        s_all = torch.empty(self.world, dtype=torch.float64, device=s_local.device)
+        dist.all_gather_into_tensor(s_all, s_local, group=self.group)
+        be.finalize(s_all)
+        be.update()
+        be.after_update(self.group)
+        return be
+
+
+class CudaRankBackend:
+    """Device side of one rank: plan, workspace, the rank's fp32 partition state and
+    reduced gradient (p elements each), its whole-model replica gradient buffer and
+    gathered half buffer (n_pad each), and IPC mappings of every peer's two buffers."""
+
+    def __init__(self, shapes: Sequence[Sequence[int]], reduce_bucket_size: int, dtype: str,
+                 rank: int, world: int, group=None, align: int = 128,
+                 scaler: Optional[ScalerCfg] = None, adamw: Optional[AdamWCfg] = None,
+                 fused_all_gather: bool = True, device: Optional[torch.device] = None):
+        self.rank, self.world, self.dtype = rank, world, dtype
+        self.device = device or torch.device("cuda", torch.cuda.current_device())
+        self.plan = Plan(shapes, world, reduce_bucket_size, align)
+        self.n_pad, self.p, self.bucket = self.plan.n_pad, self.plan.p, reduce_bucket_size
+        f32 = dict(dtype=torch.float32, device=self.device)
+        self.master = torch.zeros(self.p, **f32)
+        self.exp_avg = torch.zeros(self.p, **f32)
+        self.exp_avg_sq = torch.zeros(self.p, **f32)
+        self.reduced = torch.zeros(self.p, **f32)
+        self.grads = torch.zeros(self.n_pad, dtype=_TORCH_HALF[dtype], device=self.device)
+        self.params = torch.zeros(self.n_pad, dtype=_TORCH_HALF[dtype], device=self.device)
+        self.workspace = torch.zeros(self.plan.workspace_bytes(), dtype=torch.uint8,
+                                     device=self.device)
+        self.sumsq = torch.zeros(1, dtype=torch.float64, device=self.device)
+        self.scaler = scaler if scaler is not None else scaler_cfg(dynamic=(dtype == "fp16"))
+        self.adamw = adamw if adamw is not None else adamw_cfg()
+        self.fused_all_gather = fused_all_gather
+        zero_state_init(self.plan, self.workspace, self.scaler, self._s())
+        # peers' buffers, mapped once (IPC handles travel through the process group)
+        mine = (zero_ipc_get_handle(self.grads), zero_ipc_get_handle(self.params))
+        handles: List = [None] * world
+        dist.all_gather_object(handles, mine, group=group)
+        self._opened: List[int] = []
+        self.peer_grads, self.peer_params = [], []
+        for q in range(world):
+            if q == rank:
+                self.peer_grads.append(self.grads.data_ptr())
+                self.peer_params.append(self.params.data_ptr())
+            else:
+                g = zero_ipc_open_handle(handles[q][0])
+                p = zero_ipc_open_handle(handles[q][1])
+                self._opened += [g, p]
+                self.peer_grads.append(g)
+                self.peer_params.append(p)
+
+    def _s(self) -> int:
+        return torch.cuda.current_stream(self.device).cuda_stream
+
+    def close(self) -> None:
+        for ptr in self._opened:
+            zero_ipc_close(ptr)
+        self._opened = []
+
+    def own_slice(self) -> torch.Tensor:
+        return self.params[self.rank * self.p:(self.rank + 1) * self.p]
+
+    # ---- the step
+    def before_peer_reads(self, group) -> None:
+        # stream-ordered barrier: a rank's gradient writes precede its all-reduce, which
+        # no rank completes before all have entered it
+        flag = torch.zeros(1, device=self.device)
+        dist.all_reduce(flag, group=group)
+
+    def reduce_segment(self, b: int) -> None:
+        zero_reduce_scatter_segment(self.plan, b, self.rank, self.dtype, self.peer_grads, 0,
+                                    self.reduced, self.workspace, self._s())
+
+    def local_sumsq(self) -> torch.Tensor:
+        zero_step_local_sumsq(self.plan, self.rank, self.workspace, self.sumsq, self._s())
+        return self.sumsq
+
+    def finalize(self, s_all: torch.Tensor) -> None:
+        zero_step_finalize_ranks(self.plan, self.adamw, s_all, self.workspace, self._s())
+
+    def update(self) -> None:
+        dst = self.peer_params if self.fused_all_gather else [self.params.data_ptr()]
+        zero_step_update_partition(self.plan, self.rank, self.master, self.exp_avg,
+                                   self.exp_avg_sq, self.reduced, dst, self.dtype,
+                                   self.workspace, self._s())
+
+    def after_update(self, group) -> None:
+        if self.fused_all_gather:
+            # every rank's stores into the peers' gathered buffers have landed before any
+            # rank uses its buffer
+            flag = torch.zeros(1, device=self.device)
+            dist.all_reduce(flag, group=group)
+        else:
+            dist.all_gather_into_tensor(self.params, self.own_slice().clone(), group=group)
+
+    def result(self) -> dict:
+        return zero_get_result(self.workspace, self._s())
