@@ -140,6 +140,15 @@ typedef struct {
   int64_t adam_t;     /* applied AdamW steps so far                                  */
 } zero_step_result;
 
+/* Loss-scaler and step-counter state (what a checkpoint must keep besides the tensors). */
+typedef struct {
+  float scale;
+  int32_t cur_hysteresis;
+  int64_t iter;
+  int64_t last_overflow_iter;
+  int64_t adam_t;
+} zero_scaler_state;
+
 /* bytes per rank */
 typedef struct {
   double params, grads, optimizer_state, total;
@@ -186,6 +195,14 @@ ZERO_API int zero_workspace_bytes(const zero_plan* plan, size_t* bytes);
  * budget full. Also resets the plan's per-step bookkeeping. EINVAL on a bad config. */
 ZERO_API int zero_state_init(zero_plan* plan, void* workspace, const zero_scaler_cfg* cfg,
                     void* stream);
+/* Checkpointing ([Z2]: save through the engine so that the shard information is kept;
+ * a plain state_dict save would lose it). zero_state_read copies the scaler and step
+ * state out of the workspace (synchronises `stream`); zero_state_write installs a saved
+ * state (with its scaler configuration) into a workspace, e.g. after loading shards into
+ * a plan of another world size. */
+ZERO_API int zero_state_read(const void* workspace, zero_scaler_state* out, void* stream);
+ZERO_API int zero_state_write(zero_plan* plan, void* workspace, const zero_scaler_cfg* cfg,
+                              const zero_scaler_state* state, void* stream);
 /* Writes the half-precision copy of `master` (n_pad fp32) into the gathered buffer
  * `params` (n_pad half): round to nearest even. Used once after initialisation or a
  * load; steps keep the buffer current themselves. */

@@ -87,6 +87,15 @@ class StepResult(ctypes.Structure):
         return {f: getattr(self, f) for f, _ in self._fields_}
 
 
+class ScalerState(ctypes.Structure):
+    _fields_ = [("scale", ctypes.c_float), ("cur_hysteresis", ctypes.c_int32),
+                ("iter", ctypes.c_int64), ("last_overflow_iter", ctypes.c_int64),
+                ("adam_t", ctypes.c_int64)]
+
+    def as_dict(self) -> dict:
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
 class Memory(ctypes.Structure):
     _fields_ = [("params", ctypes.c_double), ("grads", ctypes.c_double),
                 ("optimizer_state", ctypes.c_double), ("total", ctypes.c_double)]
@@ -112,6 +121,8 @@ def _load():
         "zero_workspace_bytes": [vp, P(ctypes.c_size_t)],
         "zero_state_init": [vp, vp, P(ScalerCfg), vp],
         "zero_cast_params": [vp, vp, vp, i32, vp],
+        "zero_state_read": [vp, P(ScalerState), vp],
+        "zero_state_write": [vp, vp, P(ScalerCfg), P(ScalerState), vp],
         "zero_reduce_scatter_bucket": [vp, i64, i32, vp, i64, vp, vp, vp],
         "zero_reduce_scatter_bucket_host": [vp, i64, i32, vp, i64, vp, vp, vp, vp],
         "zero_step": [vp, P(AdamWCfg), vp, vp, vp, vp, vp, i32, vp, vp],
@@ -273,6 +284,18 @@ def adamw_cfg(lr=6e-5, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01,
 
 def zero_state_init(plan: Plan, workspace, cfg: ScalerCfg, stream=None) -> None:
     _check(lib.zero_state_init(plan.handle, _addr(workspace), ctypes.byref(cfg), _stream(stream)))
+
+
+def zero_state_read(workspace, stream=None) -> dict:
+    st = ScalerState()
+    _check(lib.zero_state_read(_addr(workspace), ctypes.byref(st), _stream(stream)))
+    return st.as_dict()
+
+
+def zero_state_write(plan: Plan, workspace, cfg: ScalerCfg, state: dict, stream=None) -> None:
+    st = ScalerState(**{k: state[k] for k, _ in ScalerState._fields_})
+    _check(lib.zero_state_write(plan.handle, _addr(workspace), ctypes.byref(cfg),
+                                ctypes.byref(st), _stream(stream)))
 
 
 def zero_cast_params(plan: Plan, master, params, param_dtype, stream=None) -> None:

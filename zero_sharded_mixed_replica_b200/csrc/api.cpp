@@ -319,6 +319,37 @@ int zero_state_init(zero_plan* plan, void* workspace, const zero_scaler_cfg* cfg
   return ZERO_OK;
 }
 
+int zero_state_read(const void* workspace, zero_scaler_state* out, void* stream) {
+  if (!workspace || !out) return fail(ZERO_EINVAL, "NULL argument");
+  WsHeader h;
+  cudaError_t e = cudaMemcpyAsync(&h, workspace, sizeof h, cudaMemcpyDeviceToHost,
+                                  (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "state copy");
+  e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  if (h.magic != kWsMagic) return fail(ZERO_ESTATE, "workspace was never initialised");
+  out->scale = h.scale;
+  out->cur_hysteresis = h.cur_hysteresis;
+  out->iter = h.iter;
+  out->last_overflow_iter = h.last_overflow_iter;
+  out->adam_t = h.adam_t;
+  return ZERO_OK;
+}
+
+int zero_state_write(zero_plan* plan, void* workspace, const zero_scaler_cfg* cfg,
+                     const zero_scaler_state* state, void* stream) {
+  if (!state) return fail(ZERO_EINVAL, "NULL argument");
+  if (!(state->scale > 0) || !isfinite(state->scale))
+    return fail(ZERO_EINVAL, "state scale must be finite and > 0");
+  if (state->iter < 0 || state->adam_t < 0 || state->adam_t > state->iter ||
+      state->last_overflow_iter < -1 || state->last_overflow_iter >= state->iter)
+    return fail(ZERO_EINVAL, "inconsistent step counters");
+  if (int rc = zero_state_init(plan, workspace, cfg, stream)) return rc;
+  cudaError_t e = launch_state_write(workspace, *state, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "state write launch");
+  return ZERO_OK;
+}
+
 int zero_cast_params(const zero_plan* plan, const float* master, void* params,
                      int32_t param_dtype, void* stream) {
   if (!plan) return fail(ZERO_EINVAL, "NULL argument");

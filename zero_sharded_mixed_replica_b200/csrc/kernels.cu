@@ -711,6 +711,19 @@ __global__ void state_init_kernel(WsHeader* h, zero_scaler_cfg cfg) {
   r.adam_t = 0;
 }
 
+__global__ void state_write_kernel(WsHeader* h, zero_scaler_state st) {
+  h->scale = st.scale;
+  h->cur_hysteresis = st.cur_hysteresis;
+  h->iter = st.iter;
+  h->last_overflow_iter = st.last_overflow_iter;
+  h->adam_t = st.adam_t;
+  h->result.scale_used = st.scale;
+  h->result.next_scale = st.scale;
+  h->result.hysteresis = st.cur_hysteresis;
+  h->result.iter = st.iter;
+  h->result.adam_t = st.adam_t;
+}
+
 // ------------------------------------------------------------------ grid sizing
 
 int sm_count() {
@@ -770,6 +783,11 @@ cudaError_t rs_grid(int64_t len, int world, int dtype, int* grid) {
 
 cudaError_t launch_state_init(void* ws, const zero_scaler_cfg& cfg, cudaStream_t s) {
   state_init_kernel<<<1, 1, 0, s>>>((WsHeader*)ws, cfg);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_state_write(void* ws, const zero_scaler_state& st, cudaStream_t s) {
+  state_write_kernel<<<1, 1, 0, s>>>((WsHeader*)ws, st);
   return cudaGetLastError();
 }
 

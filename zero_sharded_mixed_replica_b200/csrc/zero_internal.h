@@ -86,6 +86,7 @@ cudaError_t rs_grid(int64_t len, int world, int dtype, int* grid);
 
 // Launchers (kernels.cu). All return cudaSuccess or the launch error.
 cudaError_t launch_state_init(void* ws, const zero_scaler_cfg& cfg, cudaStream_t s);
+cudaError_t launch_state_write(void* ws, const zero_scaler_state& st, cudaStream_t s);
 cudaError_t launch_reduce_scatter(int world, int dtype, const uint16_t* const* g, float* R,
                                   int64_t len, double* partial, int32_t* bucket_blocks,
                                   int32_t* device_error, int grid, cudaStream_t s);
