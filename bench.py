@@ -59,6 +59,8 @@ def parse_args():
     ap.add_argument("--sweep-log2n", default="24,26,28,30")
     ap.add_argument("--sweep-world", default="1,2,4,8,16")
     ap.add_argument("--sweep-dtype", default="bf16,fp16")
+    ap.add_argument("--zero3", action="store_true",
+                    help="ZeRO-3 forward gather / release over the 7B tensor list")
     return ap.parse_args()
 
 
@@ -357,10 +359,13 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
     return out
 
 
-def run_e2e(args, wl, local_rank: int):
+def run_e2e(args, wl, local_rank: int, world_size: int = 1):
     """Same metric through the public C ABI with HOST gradient buffers: every bucket's
     replica slices are copied host -> device (pinned) inside the timed region by
-    zero_reduce_scatter_bucket_host, and the step result is read back each step."""
+    zero_reduce_scatter_bucket_host, and the step result is read back each step. Timed
+    with CUDA events on the stream that carries the copies, the kernels and the result
+    read (host waits between steps show up as idle time); max over ranks. With several
+    ranks each keeps one pinned slot (every step reuses it) to bound host memory."""
     import numpy as np
     import torch
 
@@ -383,8 +388,10 @@ def run_e2e(args, wl, local_rank: int):
     L = min(wl.bucket, plan.n_pad) if wl.streaming else plan.n_pad
     half = {"bf16": torch.bfloat16, "fp16": torch.float16}[wl.gdtype]
     # pinned host gradients: the same recipe as the device-resident run
-    host = [[torch.zeros(L, dtype=torch.int16).pin_memory() for _ in range(W)] for _ in range(2)]
-    for k in range(2):
+    n_slots = 2 if world_size == 1 else 1
+    host = [[torch.zeros(L, dtype=torch.int16).pin_memory() for _ in range(W)]
+            for _ in range(n_slots)]
+    for k in range(n_slots):
         for r in range(W):
             synthgen.grads_host(0, min(L, wl.n), wl.seed, r, wl.slot(k + 1), wl.grad_sigma,
                                 wl.spike_frac, 1.0, wl.dtype_code,
@@ -394,7 +401,7 @@ def run_e2e(args, wl, local_rank: int):
 
     def one(t):
         nonlocal h2d
-        hb = host[(t - 1) % 2]
+        hb = host[(t - 1) % n_slots]
         ptrs = [h.data_ptr() for h in hb]
         for b in range(nb):
             opt.reduce_scatter_bucket_host(b, ptrs, b * wl.bucket if wl.streaming else 0, staging)
@@ -402,14 +409,24 @@ def run_e2e(args, wl, local_rank: int):
         opt.step()
         return opt.result()  # device -> host read of the step result (synchronises)
 
+    import torch.distributed as dist
     one(1)
     torch.cuda.synchronize(dev)
+    if world_size > 1:
+        dist.barrier()
     h2d = 0
-    t0 = time.perf_counter()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
     for i in range(args.e2e_steps):
         one(i + 2)
-    dt = time.perf_counter() - t0
-    out = {"value": plan.n * args.e2e_steps / dt, "unit": "params/s",
+    e1.record(s)
+    torch.cuda.synchronize(dev)
+    dt = e0.elapsed_time(e1) / 1e3
+    if world_size > 1:
+        tt = torch.tensor([dt], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        dt = float(tt.item())
+    out = {"value": plan.n * args.e2e_steps * world_size / dt, "unit": "params/s",
            "h2d_bytes_per_step": h2d // args.e2e_steps,
            "d2h_bytes_per_step": ctypes.sizeof(zb.StepResult),
            "steps": args.e2e_steps,
@@ -477,6 +494,51 @@ def run_sweep_point(wl, steps: int, local_rank: int) -> dict:
     del opt, slots
     torch.cuda.empty_cache()
     return out
+
+
+def run_zero3_forward(args, local_rank: int) -> dict:
+    """The ZeRO-3 parameter side of a forward pass over the Llama-7B-shaped tensor list
+    (one layer per transformer block, embedding first, head last), W = 8 partitions of
+    the bf16 parameters on one GPU: every FETCH is a zero3_gather into a fresh buffer,
+    every RELEASE drops it. Knobs: max live parameters 1e9 and persistence threshold 1e6
+    as the pages configure them; the prefetch bucket the pages leave "auto" is taken as
+    the reduce bucket, 5e8. Timed with CUDA events around whole passes."""
+    import torch
+
+    import synthgen
+    import zero_sharded_mixed_replica_b200 as zb
+    from zero_sharded_mixed_replica_b200 import zero3
+
+    wl = synthgen.workload("llama7b")
+    dev = torch.device("cuda", local_rank)
+    layer_of = []
+    for t in wl.tensors:
+        if t.name.startswith("model.layers."):
+            layer_of.append(int(t.name.split(".")[2]) + 1)
+        else:
+            layer_of.append(0 if t.name.startswith("model.embed") else 33)
+    plan = zb.Plan([t.shape for t in wl.tensors], wl.world, wl.bucket, wl.align)
+    sched = zb.Zero3Schedule(plan, layer_of, 34, 500_000_000, 1_000_000_000, 1_000_000)
+    params = torch.empty(plan.n_pad, dtype=torch.bfloat16, device=dev)
+    parts = zero3.partitions_of(params, plan)
+    s = torch.cuda.current_stream(dev)
+    for _ in range(max(1, args.warmup)):
+        zero3.run_forward(plan, sched, parts, torch.bfloat16, lambda l, v: None, device=dev)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    passes = max(1, args.steps // 4)
+    for _ in range(passes):
+        zero3.run_forward(plan, sched, parts, torch.bfloat16, lambda l, v: None, device=dev)
+    e1.record(s)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / passes
+    fetched = sched.stats["fetched_elements"]
+    peak, kind = measured_peaks()
+    gbs = 4 * fetched / (ms / 1e3) / 1e9  # 2 B read + 2 B written per gathered element
+    return {"mode": "zero3_forward_gather", "workload": "llama7b_w8", "passes": passes,
+            "ms_per_forward": ms, "gathered_elements": fetched,
+            "copy_gbs": gbs, "frac_of_peak": gbs / peak, "schedule": sched.stats}
 
 
 # ---------------------------------------------------------------------------- oracle arm
@@ -565,6 +627,10 @@ def main():
             print(json.dumps(out), flush=True)
         return
 
+    if args.zero3:
+        print(json.dumps(run_zero3_forward(args, local_rank)), flush=True)
+        return
+
     if args.sweep:
         import synthgen
         for log2n in [int(x) for x in args.sweep_log2n.split(",")]:
@@ -582,12 +648,12 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     out = run_ours(args, rank, world_size, local_rank)
+    wl = get_workload(args)
+    if not args.no_e2e:
+        e2e = run_e2e(args, wl, local_rank, world_size)  # every rank takes part
+        if rank == 0:
+            out["e2e"] = e2e
     if rank == 0:
-        wl = get_workload(args)
-        if not args.no_e2e and world_size == 1:
-            out["e2e"] = run_e2e(args, wl, local_rank)
-        elif not args.no_e2e:
-            out["e2e"] = None
         if not args.no_cpu_baseline and world_size == 1:
             val, desc, steps, el = oracle_sample_run(wl, args.cpu_seconds)
             out["cpu_baseline"] = {"value": val, "unit": "params/s", "cores": 1, "kind": "oracle",

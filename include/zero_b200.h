@@ -236,6 +236,21 @@ ZERO_API int zero_reduce_scatter_bucket_host(zero_plan* plan, int64_t bucket, in
                                     int64_t host_base_offset, void* const* device_staging,
                                     float* reduced, void* workspace, void* stream);
 
+/* Gradient accumulation ([Z1] 3.1 and [Z2] config: gradient_accumulation_steps): call
+ * once per micro-batch and bucket, micro = 0 .. n_micro-1 in order. Micro-batch 0
+ * writes reduced[i] = the rank-ordered fp32 sum as zero_reduce_scatter_bucket does;
+ * each later one adds its sum: reduced[i] = reduced[i] + ((g_0[i] + g_1[i]) + ...);
+ * the last one also takes the sum of squares of the accumulated values and counts the
+ * bucket as reduced for this step. n_micro = 1 is zero_reduce_scatter_bucket. A bucket's
+ * micro-batches may interleave with other buckets' (e.g. micro-major order, bucket by
+ * bucket as backward produces them). ESTATE on a micro-batch out of order or a change of
+ * n_micro within a step. */
+ZERO_API int zero_reduce_scatter_bucket_accum(zero_plan* plan, int64_t bucket, int32_t micro,
+                                              int32_t n_micro, int32_t grad_dtype,
+                                              const void* const* replica_grads,
+                                              int64_t replica_base_offset, float* reduced,
+                                              void* workspace, void* stream);
+
 /* zero_step = zero_step_finalize + zero_step_update.
  * zero_step_finalize (one CTA): S = sum of the partial sums in a fixed order; overflow
  * = S not finite (any inf/NaN reduced gradient makes S inf or NaN); norm = sqrt(S)/scale
@@ -290,10 +305,12 @@ ZERO_API int zero_get_result(const void* workspace, zero_step_result* out, void*
  *       with an all-gather.
  *   zero_step_finalize_ranks: S = ((s_0 + s_1) + ...) + s_{W-1}, then the same scalar
  *       step as zero_step_finalize -- identical on every rank.
- *   zero_step_update_partition(r): AdamW on the local arrays; the half result goes to
- *       params_dst[d] + r*p for every d -- this rank's own gathered buffer and, mapped
- *       over CUDA IPC, its peers' (the all-gather fused into the update as P2P stores),
- *       or only its own when the caller all-gathers afterwards.
+ *   zero_step_update_partition(r): AdamW on the local arrays; the p half results go to
+ *       params_dst[d][0 .. p) for every d: where rank r's slice lives in each
+ *       destination -- gathered buffer + r*p of this rank and, mapped over CUDA IPC, of
+ *       its peers (the all-gather fused into the update as P2P stores), or a buffer
+ *       holding only this rank's partition (parameters partitioned as in ZeRO-3).
+ *       Each destination must be 16-byte aligned (choose align so that p*2 % 16 == 0).
  * Errors as above; ESTATE when a segment is reduced twice, a bucket outside the rank's
  * partition is reduced, or the calls come out of order. */
 ZERO_API int zero_reduce_scatter_segment(zero_plan* plan, int64_t bucket, int32_t rank,
@@ -317,6 +334,62 @@ ZERO_API int zero_ipc_handle_bytes(void);
 ZERO_API int zero_ipc_get_handle(const void* device_ptr, void* handle_out);
 ZERO_API int zero_ipc_open_handle(const void* handle, void** device_ptr);
 ZERO_API int zero_ipc_close(void* device_ptr);
+
+/* ---------------------------------------------------------------- ZeRO-3 parameters
+ * Stage 3 partitions the half parameters too ([Z1] 1.2.3; [Z2]; [Z3] technical insight):
+ * rank r keeps only its partition (p halves; the update writes it with
+ * zero_step_update_partition or, on one GPU, into slice r of the gathered buffer), and
+ * a layer's tensors are all-gathered before its forward pass and dropped after it.
+ *
+ * zero3_schedule_create: the fetch / release order for a forward pass over n_layers
+ * layers run in order (layer_of_tensor[t] in [0, n_layers), or -1 for a tensor the
+ * forward pass does not use), from the knobs of [Z1] 3.1 / 6:
+ *   - tensors with numel <= persistence_threshold (stage3_param_persistence_threshold)
+ *     are fetched once, first, and never released;
+ *   - before layer i: FETCH its tensors that are not live (even past the budget);
+ *   - then prefetch the later layers' tensors in order while the live elements fetched
+ *     ahead of layer i stay <= prefetch_bucket_size (stage3_prefetch_bucket_size) and
+ *     all live elements stay <= max_live_parameters (stage3_max_live_parameters); the
+ *     first tensor that does not fit stops the prefetch; the prefetched tensors form one
+ *     FETCH (one bucketed all-gather);
+ *   - COMPUTE layer i, then RELEASE its tensors.
+ * Events reference runs of the tensor-id list (zero3_schedule_tensors). */
+#define ZERO3_FETCH 0
+#define ZERO3_COMPUTE 1
+#define ZERO3_RELEASE 2
+typedef struct zero3_schedule zero3_schedule; /* opaque, host memory */
+typedef struct {
+  int32_t op;    /* ZERO3_FETCH / ZERO3_COMPUTE / ZERO3_RELEASE                        */
+  int32_t layer; /* the layer being run (-1: the persistent fetch before layer 0)       */
+  int64_t first; /* first index into the tensor-id list                                 */
+  int64_t count; /* tensor ids in this event                                            */
+} zero3_event;
+typedef struct {
+  int64_t peak_live_elements;  /* live half elements at the busiest compute, persistent included */
+  int64_t fetched_elements;    /* elements all-gathered over the forward pass                    */
+  int64_t fetch_events;        /* bucketed all-gathers                                            */
+  int64_t persistent_elements; /* elements kept for the whole pass                                */
+  int64_t over_budget_layers;  /* layers whose own tensors exceeded max_live_parameters           */
+} zero3_stats;
+ZERO_API int zero3_schedule_create(const zero_plan* plan, const int32_t* layer_of_tensor,
+                                   int32_t n_layers, int64_t prefetch_bucket_size,
+                                   int64_t max_live_parameters, int64_t persistence_threshold,
+                                   zero3_schedule** out);
+ZERO_API int zero3_schedule_events(const zero3_schedule* s, zero3_event* out, int64_t cap,
+                                   int64_t* count);
+ZERO_API int zero3_schedule_tensors(const zero3_schedule* s, int32_t* out, int64_t cap,
+                                    int64_t* count);
+ZERO_API int zero3_schedule_stats(const zero3_schedule* s, zero3_stats* out);
+ZERO_API void zero3_schedule_destroy(zero3_schedule* s);
+
+/* zero3_gather: the all-gather of a FETCH. dst receives the listed tensors' half values
+ * back to back, in the order given; element i of the flat space is read from
+ * partitions[i / p][i % p] (partitions[r]: rank r's partition of p halves -- peer memory
+ * mapped over CUDA IPC in a multi-process run, read over NVLink; slices of the gathered
+ * buffer on one GPU). One launch for up to 64 contiguous pieces, 16-byte vector copies
+ * where source and destination share their alignment. */
+ZERO_API int zero3_gather(const zero_plan* plan, const int32_t* tensors, int32_t n_tensors,
+                          const void* const* partitions, void* dst, void* stream);
 
 /* ---------------------------------------------------------------- no-alloc variant
  * zero_reduce_sumsq_noalloc has no counterpart in the pages. It is for callers that
@@ -345,6 +418,13 @@ ZERO_API int zero_ipc_close(void* device_ptr);
 ZERO_API int zero_reduce_sumsq_noalloc(int32_t world_size, int32_t grad_dtype,
                                        const void* const* replica_grads, int64_t n,
                                        float* reduced, double* sumsq, void* stream);
+
+/* Diagnostics: launches one thread that waits on a barrier phase nothing completes, so
+ * the kernels' bounded wait (about one second) runs out; it records its code (64) in the
+ * workspace's sticky device_error, as a pipeline wait that gave up would. The next
+ * zero_get_result then returns ZERO_EDEVICE and the CUDA context stays usable;
+ * zero_state_init clears the flag. */
+ZERO_API int zero_selftest_bounded_wait(void* workspace, void* stream);
 
 ZERO_API const char* zero_last_error(void);
 ZERO_API int zero_abi_version(void);

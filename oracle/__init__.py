@@ -106,6 +106,7 @@ def lib():
         L.oracle_half_to_f32_array.argtypes = [vp, vp, i64, i32]
         L.oracle_state_init.argtypes = [ctypes.POINTER(ScalerCfg), ctypes.POINTER(State)]
         L.oracle_reduce.argtypes = [i32, i32, vp, i64, vp]
+        L.oracle_reduce_accumulate.argtypes = [i32, i32, vp, i64, vp]
         L.oracle_sumsq.argtypes = [vp, i64, ctypes.POINTER(ctypes.c_double)]
         L.oracle_any_nonfinite.restype = i32
         L.oracle_any_nonfinite.argtypes = [vp, i64]
@@ -224,6 +225,10 @@ def reduce(grads: Sequence[np.ndarray], dtype: int) -> np.ndarray:
     return R
 
 
+def reduce_accumulate(grads: Sequence[np.ndarray], dtype: int, R: np.ndarray) -> None:
+    lib().oracle_reduce_accumulate(len(grads), dtype, _ptr_array(grads), grads[0].size, _ptr(R))
+
+
 def sumsq(R: np.ndarray, S: float = 0.0) -> float:
     acc = ctypes.c_double(S)
     lib().oracle_sumsq(_ptr(R), R.size, ctypes.byref(acc))
@@ -309,23 +314,27 @@ def step_grad_scale(wl, st: State) -> float:
 
 
 def resident_grads(wl, n_pad: int, t: int, scale: float,
-                   out: Optional[List[np.ndarray]] = None) -> List[np.ndarray]:
-    """Replica gradients of step t over the whole padded space (input recipe)."""
+                   out: Optional[List[np.ndarray]] = None, micro: int = 0) -> List[np.ndarray]:
+    """Replica gradients of step t (micro-batch `micro`) over the whole padded space
+    (input recipe); +inf sites go into the step's last micro-batch."""
     dt = wl.dtype_code
     if out is None:
         out = [np.zeros(n_pad, np.uint16) for _ in range(wl.world)]
     for r in range(wl.world):
-        synthgen.grads_host(0, wl.n, wl.seed, r, wl.slot(t), wl.grad_sigma, wl.spike_frac,
-                            scale, dt, out=out[r][:wl.n])
+        synthgen.grads_host(0, wl.n, wl.seed, r, wl.micro_slot(t, micro), wl.grad_sigma,
+                            wl.spike_frac, scale, dt, out=out[r][:wl.n])
         out[r][wl.n:] = 0
-    inf = np.uint16(0x7c00 if dt == FP16 else 0x7f80)
-    for idx, rep in wl.inf_sites_at(t):
-        out[rep][idx] = inf
+    if micro == wl.micro_batches - 1:
+        inf = np.uint16(0x7c00 if dt == FP16 else 0x7f80)
+        for idx, rep in wl.inf_sites_at(t):
+            out[rep][idx] = inf
     return out
 
 
 def run_resident(wl, steps: Optional[int] = None, on_step=None) -> dict:
-    """All steps of a resident workload on the full arrays; returns final state."""
+    """All steps of a resident workload on the full arrays; returns final state. With
+    micro_batches > 1 the reduced gradient accumulates over the micro-batches of a step
+    (bucket by bucket, in micro-batch order) before the norm is taken."""
     pl = plan(wl.numels, wl.world, wl.bucket, wl.align)
     cfg, hp = workload_cfg(wl)
     st = state_init(cfg)
@@ -338,8 +347,24 @@ def run_resident(wl, steps: Optional[int] = None, on_step=None) -> dict:
     grads = None
     scalars = []
     for t in range(1, (steps or wl.steps) + 1):
-        grads = resident_grads(wl, pl.n_pad, t, step_grad_scale(wl, st), out=grads)
-        sc = step(grads, dt, wl.bucket, R, master, m, v, params, dt, cfg, hp, st)
+        scale = step_grad_scale(wl, st)
+        if wl.micro_batches == 1:
+            grads = resident_grads(wl, pl.n_pad, t, scale, out=grads)
+            sc = step(grads, dt, wl.bucket, R, master, m, v, params, dt, cfg, hp, st)
+        else:
+            for k in range(wl.micro_batches):
+                grads = resident_grads(wl, pl.n_pad, t, scale, out=grads, micro=k)
+                if k == 0:
+                    R[:] = reduce(grads, dt)
+                else:
+                    reduce_accumulate(grads, dt, R)
+            S, bad = 0.0, False
+            for b in range(pl.n_buckets):
+                s0, ln = pl.bucket_range(b)
+                S = S + sumsq(R[s0:s0 + ln])
+                bad = bad or any_nonfinite(R[s0:s0 + ln])
+            sc = finalize(S, bad, cfg, hp, st)
+            adamw(R, master, m, v, params, dt, sc)
         scalars.append(sc.as_dict())
         if on_step is not None:
             on_step(t, sc, R, master, m, v, params)

@@ -202,6 +202,15 @@ void oracle_reduce(int32_t world, int32_t gdtype, const uint16_t* const* grads, 
   }
 }
 
+void oracle_reduce_accumulate(int32_t world, int32_t gdtype, const uint16_t* const* grads,
+                              int64_t n, float* R) {
+  for (int64_t i = 0; i < n; ++i) {
+    float acc = oracle_half_to_f32(grads[0][i], gdtype);
+    for (int32_t r = 1; r < world; ++r) acc = acc + oracle_half_to_f32(grads[r][i], gdtype);
+    R[i] = R[i] + acc;
+  }
+}
+
 void oracle_sumsq(const float* R, int64_t n, double* S) {
   double acc = *S;
   for (int64_t i = 0; i < n; ++i) {

@@ -113,6 +113,13 @@ void oracle_state_init(const oracle_scaler_cfg* cfg, oracle_state* st);
 void oracle_reduce(int32_t world, int32_t gdtype, const uint16_t* const* grads, int64_t n,
                    float* R);
 
+/* Gradient accumulation over micro-batches ([Z1] 3.1 and [Z2] config:
+ * gradient_accumulation_steps): R[i] = R[i] + (((g_0[i] + g_1[i]) + ...) + g_{W-1}[i]),
+ * the micro-batch's rank-ordered fp32 sum added to what the earlier micro-batches of
+ * the step left in R. */
+void oracle_reduce_accumulate(int32_t world, int32_t gdtype, const uint16_t* const* grads,
+                              int64_t n, float* R);
+
 /* S += R[0]^2 + R[1]^2 + ... in flat order, each square formed in fp64. */
 void oracle_sumsq(const float* R, int64_t n, double* S);
 

@@ -16,6 +16,8 @@ Recipe (values are pure functions of seed, stream, step slot and index; see
     streaming workloads: the W replica buffers hold one bucket; buffer index =
     flat index - bucket start, slot = (t - 1) % 2.
   * +inf injection: site k of step t picks a flat index in [0, N) and a replica.
+  * gradient accumulation (M micro-batches per step, resident workloads): micro-batch k
+    of step t draws slot (t-1)*M + k + 1; +inf sites go into the last micro-batch.
 """
 from __future__ import annotations
 
@@ -256,6 +258,7 @@ class Workload:
     eps: float = 1e-8
     weight_decay: float = 0.01
     max_grad_norm: float = 1.0
+    micro_batches: int = 1        # gradient accumulation steps per optimizer step
 
     @property
     def numels(self) -> List[int]:
@@ -271,6 +274,11 @@ class Workload:
 
     def slot(self, t: int) -> int:
         return (t - 1) % 2 if self.streaming else t
+
+    def micro_slot(self, t: int, k: int) -> int:
+        """Slot of micro-batch k of step t (resident workloads): (t-1)*M + k + 1, which
+        is the step number t when there is one micro-batch."""
+        return (t - 1) * self.micro_batches + k + 1 if self.micro_batches > 1 else self.slot(t)
 
     def grad_buffer_len(self, n_pad: int) -> int:
         return min(self.bucket, n_pad) if self.streaming else n_pad

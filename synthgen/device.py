@@ -23,10 +23,12 @@ def init_master(wl, master: torch.Tensor, stream: int) -> None:
 
 
 def fill_grads(wl, bufs: Sequence[torch.Tensor], j0: int, n: int, t: int, scale: float,
-               stream: int) -> None:
-    """bufs[r][0:n] <- replica r's gradient bits at buffer indices j0 .. j0+n-1, step t."""
+               stream: int, micro: int = 0) -> None:
+    """bufs[r][0:n] <- replica r's gradient bits at buffer indices j0 .. j0+n-1, step t
+    (micro-batch `micro` of a resident workload with gradient accumulation)."""
+    slot = wl.micro_slot(t, micro) if not wl.streaming else wl.slot(t)
     for r, b in enumerate(bufs):
-        grads_cuda(b.data_ptr(), j0, n, wl.seed, r, wl.slot(t), wl.grad_sigma, wl.spike_frac,
+        grads_cuda(b.data_ptr(), j0, n, wl.seed, r, slot, wl.grad_sigma, wl.spike_frac,
                    scale, wl.dtype_code, stream)
 
 

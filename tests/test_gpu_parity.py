@@ -401,3 +401,63 @@ def test_sweep_2_30_w16_sampled():
                                     [b * wl.bucket + d for b in range(1, 6) for d in (-1, 0)],
                                     [r * (n // 16) + d for r in range(1, 16) for d in (-1, 0)]]))
     _check_streaming(wl, idx.astype(np.int64))
+
+
+# ----------------------------------------------------------------------------- accumulation
+
+@pytest.mark.parametrize("dtype,W,M", [("bf16", 8, 4), ("fp16", 4, 3)])
+def test_gradient_accumulation(dtype, W, M):
+    """M micro-batches per step, reduced bucket by bucket in micro-major order and
+    accumulated in the fp32 reduced gradient; fp16 with a +inf in step 2's last
+    micro-batch (the whole step is skipped)."""
+    t = synthgen.TensorSpec
+    wl = synthgen.Workload("accum", [t("a", (300007,), "normal"), t("b", (64, 33), "ones")],
+                           world=W, bucket=100000, steps=3, gdtype=dtype,
+                           dynamic=dtype == "fp16", align=8, grad_sigma=1e-2,
+                           inf_sites={2: 1} if dtype == "fp16" else {}, micro_batches=M)
+    ref = oracle.run_resident(wl)
+    opt = make_opt(wl)
+    s = stream()
+    sdev.init_master(wl, opt.master, s)
+    opt.cast_params()
+    n_pad = opt.plan.n_pad
+    grads = [torch.zeros(n_pad, dtype=HALF[dtype], device="cuda") for _ in range(W)]
+    scale = float(2.0 ** wl.init_scale_power) if wl.dynamic else 1.0
+    for step in range(1, wl.steps + 1):
+        for k in range(M):
+            sdev.fill_grads(wl, grads, 0, wl.n, step, scale, s, micro=k)
+            if k == M - 1:
+                sdev.plant_infs(wl, grads, step)
+            for b in range(opt.plan.n_buckets):
+                opt.reduce_scatter_bucket_accum(b, k, M, grads)
+        opt.step()
+        res = opt.result()
+        check_scalars(res, ref["scalars"][step - 1])
+        scale = float(res["next_scale"]) if wl.dynamic else 1.0
+    if dtype == "fp16":
+        assert [s_["skipped"] for s_ in ref["scalars"]] == [0, 1, 0]
+    check_all(opt, ref, W)
+    # out of order: micro-batch 1 before 0
+    with pytest.raises(zb.ZeroError) as e:
+        opt.reduce_scatter_bucket_accum(0, 1, M, grads)
+    assert e.value.code == zb.ZERO_ESTATE
+
+
+# ----------------------------------------------------------------------------- bounded waits
+
+def test_bounded_wait_gives_up_and_reports():
+    """A wait that nothing completes ends after about a second with the sticky error
+    flag set; zero_get_result reports ZERO_EDEVICE, the context stays usable, and a
+    state re-initialisation clears the flag."""
+    import time
+    opt = zb.ZeroOptimizer([(4096,)], 2, 4096)
+    t0 = time.perf_counter()
+    zb.zero_selftest_bounded_wait(opt.workspace)
+    with pytest.raises(zb.ZeroError) as e:
+        opt.result()
+    assert e.value.code == zb.ZERO_EDEVICE
+    assert 0.5 < time.perf_counter() - t0 < 30
+    zb.zero_state_init(opt.plan, opt.workspace, opt.scaler)
+    g = [torch.zeros(opt.plan.n_pad, dtype=torch.bfloat16, device="cuda")] * 2
+    opt.full_step(g)
+    assert opt.result()["device_error"] == 0

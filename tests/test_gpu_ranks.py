@@ -79,7 +79,7 @@ def test_rank_local_calls_match_oracle(case):
         for r, rk in enumerate(ranks):
             zb.zero_step_finalize_ranks(rk["plan"], adamw, s_all, rk["ws"], s)
             zb.zero_step_update_partition(rk["plan"], r, rk["master"], rk["m"], rk["v"], rk["R"],
-                                          gathered, wl.gdtype, rk["ws"], s)
+                                          [g[r * p:] for g in gathered], wl.gdtype, rk["ws"], s)
             results.append(zb.zero_get_result(rk["ws"], s))
         sc = ref["scalars"][t - 1] if t == wl.steps else None
         # every rank decided the same

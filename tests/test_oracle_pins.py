@@ -435,3 +435,36 @@ def test_memory_accounting_matches_pages():
     for W in (1, 2, 8, 64):
         tot = [oracle.memory_per_rank(psi, W, s)["total"] for s in range(4)]
         assert tot == sorted(tot, reverse=True)
+
+
+# ----------------------------------------------------------------------------- accumulation
+
+def test_accumulation_exact_and_ordered():
+    # dyadic micro-batch gradients: the accumulated fp32 sum is the exact integer sum
+    rng = np.random.default_rng(9)
+    W, n, M = 4, 2048, 5
+    ints = rng.integers(-100, 101, (M, W, n))
+    R = oracle.reduce([_bf16((ints[0, r] / 512.0).tolist()) for r in range(W)], BF16)
+    for k in range(1, M):
+        oracle.reduce_accumulate([_bf16((ints[k, r] / 512.0).tolist()) for r in range(W)], BF16, R)
+    assert np.array_equal(R.astype(np.float64), ints.sum((0, 1)) / 512.0)
+    # micro-batch order is kept: R = 2^24, then + (1), then + (-2^24) gives 0, while
+    # (2^24) + (1 - 2^24 within one micro-batch) gives 1 -- one fp32 add per micro-batch
+    a, b, c = 2.0 ** 24, 1.0, -(2.0 ** 24)
+    R = oracle.reduce([_bf16([a, a])], BF16)
+    oracle.reduce_accumulate([_bf16([b, b])], BF16, R)
+    oracle.reduce_accumulate([_bf16([c, 0.0])], BF16, R)
+    assert R.tolist() == [0.0, 2.0 ** 24]
+    R2 = oracle.reduce([_bf16([a])], BF16)
+    oracle.reduce_accumulate([_bf16([b]), _bf16([c])], BF16, R2)
+    assert R2.tolist() == [1.0]
+
+
+def test_one_micro_batch_is_the_plain_step():
+    wl = synthgen.workload("tiny")
+    a = oracle.run_resident(wl, steps=2)
+    wl2 = synthgen.workload("tiny")
+    wl2.micro_batches = 1
+    b = oracle.run_resident(wl2, steps=2)
+    for k in ("master", "m", "v", "params", "R"):
+        assert np.array_equal(a[k], b[k])

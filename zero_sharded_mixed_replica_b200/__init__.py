@@ -96,6 +96,17 @@ class ScalerState(ctypes.Structure):
         return {f: getattr(self, f) for f, _ in self._fields_}
 
 
+class Zero3Event(ctypes.Structure):
+    _fields_ = [("op", ctypes.c_int32), ("layer", ctypes.c_int32), ("first", ctypes.c_int64),
+                ("count", ctypes.c_int64)]
+
+
+class Zero3Stats(ctypes.Structure):
+    _fields_ = [("peak_live_elements", ctypes.c_int64), ("fetched_elements", ctypes.c_int64),
+                ("fetch_events", ctypes.c_int64), ("persistent_elements", ctypes.c_int64),
+                ("over_budget_layers", ctypes.c_int64)]
+
+
 class Memory(ctypes.Structure):
     _fields_ = [("params", ctypes.c_double), ("grads", ctypes.c_double),
                 ("optimizer_state", ctypes.c_double), ("total", ctypes.c_double)]
@@ -125,6 +136,7 @@ def _load():
         "zero_state_write": [vp, vp, P(ScalerCfg), P(ScalerState), vp],
         "zero_reduce_scatter_bucket": [vp, i64, i32, vp, i64, vp, vp, vp],
         "zero_reduce_scatter_bucket_host": [vp, i64, i32, vp, i64, vp, vp, vp, vp],
+        "zero_reduce_scatter_bucket_accum": [vp, i64, i32, i32, i32, vp, i64, vp, vp, vp],
         "zero_step": [vp, P(AdamWCfg), vp, vp, vp, vp, vp, i32, vp, vp],
         "zero_step_finalize": [vp, P(AdamWCfg), vp, vp],
         "zero_step_update": [vp, vp, vp, vp, vp, vp, i32, vp, vp],
@@ -139,6 +151,13 @@ def _load():
         "zero_ipc_open_handle": [vp, P(vp)],
         "zero_ipc_close": [vp],
         "zero_reduce_sumsq_noalloc": [i32, i32, vp, i64, vp, vp, vp],
+        "zero_selftest_bounded_wait": [vp, vp],
+        "zero3_schedule_create": [vp, vp, i32, i64, i64, i64, P(vp)],
+        "zero3_schedule_events": [vp, vp, i64, P(i64)],
+        "zero3_schedule_tensors": [vp, vp, i64, P(i64)],
+        "zero3_schedule_stats": [vp, P(Zero3Stats)],
+        "zero3_schedule_destroy": [vp],
+        "zero3_gather": [vp, vp, i32, vp, vp, vp],
         "zero_last_error": [],
         "zero_abi_version": [],
     }
@@ -147,6 +166,7 @@ def _load():
         fn.argtypes = args
         fn.restype = ctypes.c_int
     L.zero_plan_destroy.restype = None
+    L.zero3_schedule_destroy.restype = None
     L.zero_last_error.restype = ctypes.c_char_p
     return L
 
@@ -320,6 +340,15 @@ def zero_reduce_scatter_bucket_host(plan: Plan, bucket: int, grad_dtype,
         _stream(stream)))
 
 
+def zero_reduce_scatter_bucket_accum(plan: Plan, bucket: int, micro: int, n_micro: int,
+                                     grad_dtype, replica_grads: Sequence,
+                                     replica_base_offset: int, reduced, workspace,
+                                     stream=None) -> None:
+    _check(lib.zero_reduce_scatter_bucket_accum(
+        plan.handle, bucket, micro, n_micro, _dtype(grad_dtype), _ptr_array(replica_grads),
+        int(replica_base_offset), _addr(reduced), _addr(workspace), _stream(stream)))
+
+
 def zero_step(plan: Plan, cfg: AdamWCfg, master, exp_avg, exp_avg_sq, reduced, params,
               param_dtype, workspace, stream=None) -> None:
     _check(lib.zero_step(plan.handle, ctypes.byref(cfg), _addr(master), _addr(exp_avg),
@@ -349,6 +378,55 @@ def zero_get_result(workspace, stream=None) -> dict:
     r = StepResult()
     _check(lib.zero_get_result(_addr(workspace), ctypes.byref(r), _stream(stream)))
     return r.as_dict()
+
+
+def zero_selftest_bounded_wait(workspace, stream=None) -> None:
+    _check(lib.zero_selftest_bounded_wait(_addr(workspace), _stream(stream)))
+
+
+ZERO3_FETCH, ZERO3_COMPUTE, ZERO3_RELEASE = 0, 1, 2
+
+
+class Zero3Schedule:
+    """The ZeRO-3 fetch / compute / release order of one forward pass (host memory)."""
+
+    def __init__(self, plan: Plan, layer_of_tensor: Sequence[int], n_layers: int,
+                 prefetch_bucket_size: int, max_live_parameters: int,
+                 persistence_threshold: int):
+        arr = (ctypes.c_int32 * max(len(layer_of_tensor), 1))(*layer_of_tensor)
+        h = ctypes.c_void_p()
+        _check(lib.zero3_schedule_create(plan.handle, arr, n_layers, int(prefetch_bucket_size),
+                                         int(max_live_parameters), int(persistence_threshold),
+                                         ctypes.byref(h)))
+        self._h = h
+        self._destroy = lib.zero3_schedule_destroy
+        cnt = ctypes.c_int64()
+        _check(lib.zero3_schedule_events(h, None, 0, ctypes.byref(cnt)))
+        ev = (Zero3Event * max(cnt.value, 1))()
+        _check(lib.zero3_schedule_events(h, ev, cnt.value, ctypes.byref(cnt)))
+        tc = ctypes.c_int64()
+        _check(lib.zero3_schedule_tensors(h, None, 0, ctypes.byref(tc)))
+        ts = (ctypes.c_int32 * max(tc.value, 1))()
+        _check(lib.zero3_schedule_tensors(h, ts, tc.value, ctypes.byref(tc)))
+        ids = list(ts[:tc.value])
+        self.events = [(e.op, e.layer, ids[e.first:e.first + e.count]) for e in ev[:cnt.value]]
+        st = Zero3Stats()
+        _check(lib.zero3_schedule_stats(h, ctypes.byref(st)))
+        self.stats = {f: getattr(st, f) for f, _ in Zero3Stats._fields_}
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        d = getattr(self, "_destroy", None)
+        if h is not None and h.value and d is not None:
+            d(h)
+            self._h = None
+
+
+def zero3_gather(plan: Plan, tensors: Sequence[int], partitions: Sequence, dst,
+                 stream=None) -> None:
+    arr = (ctypes.c_int32 * max(len(tensors), 1))(*tensors)
+    _check(lib.zero3_gather(plan.handle, arr, len(tensors), _ptr_array(partitions) if partitions else None,
+                            _addr(dst), _stream(stream)))
 
 
 def zero_abi_version() -> int:

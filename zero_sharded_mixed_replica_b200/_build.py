@@ -5,7 +5,7 @@ import subprocess
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB_PATH = os.path.join(PKG, "libzero_b200.so")
-SOURCES = [os.path.join(PKG, "csrc", f) for f in ("api.cpp", "kernels.cu", "noalloc.cu")]
+SOURCES = [os.path.join(PKG, "csrc", f) for f in ("api.cpp", "kernels.cu", "noalloc.cu", "zero3.cpp", "zero3_gather.cu")]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "-Xcompiler", "-fPIC,-fvisibility=hidden", "-shared"]
 

@@ -54,7 +54,8 @@ int check_adamw(const zero_adamw_cfg* c) {
 
 // K1 for bucket b with replica pointers already checked
 int reduce_bucket(zero_plan* plan, int64_t b, int32_t dt, const uint16_t* const* g_at_start,
-                  float* reduced, void* ws, cudaStream_t s) {
+                  float* reduced, void* ws, cudaStream_t s, int accumulate = 0,
+                  int want_sumsq = 1) {
   const int64_t start = b * plan->bucket, len = bucket_len(plan, b);
   int grid = 1;
   cudaError_t e = rs_grid(len, plan->world, dt, &grid);
@@ -62,10 +63,13 @@ int reduce_bucket(zero_plan* plan, int64_t b, int32_t dt, const uint16_t* const*
   e = launch_reduce_scatter(plan->world, dt, g_at_start, reduced + start, len,
                             ws_partial(plan, ws) + b * plan->slots_full,
                             ws_bucket_blocks(plan, ws) + b,
-                            &((WsHeader*)ws)->result.device_error, grid, s);
+                            &((WsHeader*)ws)->result.device_error, grid, s, accumulate,
+                            want_sumsq);
   if (e != cudaSuccess) return cuda_fail(e, "reduce-scatter launch");
-  plan->reduced[b] = 1;
-  plan->reduced_count += 1;
+  if (want_sumsq) {
+    plan->reduced[b] = 1;
+    plan->reduced_count += 1;
+  }
   return ZERO_OK;
 }
 
@@ -177,6 +181,7 @@ int zero_plan_create(const int64_t* dims, const int32_t* ndims, int32_t n_tensor
     p->slots_last = p->n_buckets ? rs_slots(bucket_len(p, p->n_buckets - 1)) : 0;
     p->total_slots = p->n_buckets ? (p->n_buckets - 1) * p->slots_full + p->slots_last : 0;
     p->reduced.assign((size_t)p->n_buckets, 0);
+    p->next_micro.assign((size_t)p->n_buckets, 0);
     p->ws_bucket_blocks_off = kWsHeaderBytes;
     p->ws_partial_off =
         round_up(p->ws_bucket_blocks_off + sizeof(int32_t) * (size_t)p->n_buckets, 256);
@@ -315,6 +320,8 @@ int zero_state_init(zero_plan* plan, void* workspace, const zero_scaler_cfg* cfg
   if (e != cudaSuccess) return cuda_fail(e, "state init launch");
   plan->reduced.assign((size_t)plan->n_buckets, 0);
   plan->reduced_count = 0;
+  plan->next_micro.assign((size_t)plan->n_buckets, 0);
+  plan->n_micro = 0;
   plan->finalized = false;
   return ZERO_OK;
 }
@@ -407,6 +414,39 @@ int zero_reduce_scatter_bucket_host(zero_plan* plan, int64_t bucket, int32_t gra
   return reduce_bucket(plan, bucket, grad_dtype, g, reduced, workspace, (cudaStream_t)stream);
 }
 
+int zero_reduce_scatter_bucket_accum(zero_plan* plan, int64_t bucket, int32_t micro,
+                                     int32_t n_micro, int32_t grad_dtype,
+                                     const void* const* replica_grads,
+                                     int64_t replica_base_offset, float* reduced,
+                                     void* workspace, void* stream) {
+  if (int rc = check_bucket_call(plan, bucket, grad_dtype, reduced, workspace)) return rc;
+  if (!replica_grads) return fail(ZERO_EINVAL, "replica_grads is NULL");
+  if (n_micro < 1) return fail(ZERO_EINVAL, "n_micro must be >= 1");
+  if (plan->n_micro != 0 && plan->n_micro != n_micro)
+    return fail(ZERO_ESTATE, "n_micro changed within a step");
+  if (micro != plan->next_micro[bucket])
+    return fail(ZERO_ESTATE, "micro-batch " + std::to_string(micro) + " of bucket " +
+                                 std::to_string(bucket) + " out of order (expected " +
+                                 std::to_string(plan->next_micro[bucket]) + ")");
+  const int64_t start = bucket * plan->bucket;
+  if (replica_base_offset < 0 || replica_base_offset > start)
+    return fail(ZERO_EINVAL, "replica_base_offset must be in [0, bucket start]");
+  const uint16_t* g[ZERO_MAX_WORLD];
+  for (int r = 0; r < plan->world; ++r) {
+    if (!replica_grads[r]) return fail(ZERO_EINVAL, "replica_grads[" + std::to_string(r) + "] is NULL");
+    if (!aligned16(replica_grads[r]))
+      return fail(ZERO_EALIGN, "replica_grads[" + std::to_string(r) + "] is not 16-byte aligned");
+    g[r] = (const uint16_t*)replica_grads[r] + (start - replica_base_offset);
+  }
+  const bool last = micro == n_micro - 1;
+  if (int rc = reduce_bucket(plan, bucket, grad_dtype, g, reduced, workspace,
+                             (cudaStream_t)stream, micro > 0 ? 1 : 0, last ? 1 : 0))
+    return rc;
+  plan->n_micro = n_micro;
+  plan->next_micro[bucket] = last ? 0 : micro + 1;
+  return ZERO_OK;
+}
+
 int zero_step_finalize(zero_plan* plan, const zero_adamw_cfg* cfg, void* workspace,
                        void* stream) {
   if (!plan || !workspace) return fail(ZERO_EINVAL, "NULL argument");
@@ -422,6 +462,8 @@ int zero_step_finalize(zero_plan* plan, const zero_adamw_cfg* cfg, void* workspa
   if (e != cudaSuccess) return cuda_fail(e, "finalize launch");
   plan->reduced.assign((size_t)plan->n_buckets, 0);
   plan->reduced_count = 0;
+  plan->next_micro.assign((size_t)plan->n_buckets, 0);
+  plan->n_micro = 0;
   plan->finalized = true;
   return ZERO_OK;
 }
@@ -580,6 +622,8 @@ int zero_step_finalize_ranks(zero_plan* plan, const zero_adamw_cfg* cfg,
   if (e != cudaSuccess) return cuda_fail(e, "finalize launch");
   plan->reduced.assign((size_t)plan->n_buckets, 0);
   plan->reduced_count = 0;
+  plan->next_micro.assign((size_t)plan->n_buckets, 0);
+  plan->n_micro = 0;
   plan->local_summed = false;
   plan->finalized = true;
   return ZERO_OK;
@@ -603,10 +647,9 @@ int zero_step_update_partition(zero_plan* plan, int32_t rank, float* master_loca
   void* dst[ZERO_MAX_WORLD];
   for (int d = 0; d < n_dst; ++d) {
     if (!params_dst[d] && plan->p > 0) return fail(ZERO_EINVAL, "params_dst has a NULL entry");
-    // this rank's slice of each gathered buffer
-    dst[d] = (uint16_t*)params_dst[d] + (int64_t)rank * plan->p;
+    dst[d] = params_dst[d];  // where this rank's p half values go in destination d
     if (!aligned16(dst[d]))
-      return fail(ZERO_EALIGN, "params_dst[" + std::to_string(d) + "] + rank*p is not 16-byte aligned");
+      return fail(ZERO_EALIGN, "params_dst[" + std::to_string(d) + "] is not 16-byte aligned");
   }
   if (!plan->finalized)
     return fail(ZERO_ESTATE, "zero_step_update_partition without a finalize before it");
@@ -615,6 +658,16 @@ int zero_step_update_partition(zero_plan* plan, int32_t rank, float* master_loca
                                 (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "update launch");
   plan->finalized = false;
+  return ZERO_OK;
+}
+
+// ------------------------------------------------------------------ diagnostics
+
+int zero_selftest_bounded_wait(void* workspace, void* stream) {
+  if (!workspace) return fail(ZERO_EINVAL, "NULL argument");
+  if (!aligned16(workspace)) return fail(ZERO_EALIGN, "workspace must be 16-byte aligned");
+  cudaError_t e = launch_selftest_wait(workspace, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
   return ZERO_OK;
 }
 

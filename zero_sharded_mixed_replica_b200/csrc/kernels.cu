@@ -37,6 +37,15 @@ __device__ __forceinline__ float4 ld_nc_f4(const float* p) {
   return r;
 }
 
+// coherent load for data this kernel later overwrites at the same address
+__device__ __forceinline__ float4 ld_f4(const float* p) {
+  float4 r;
+  asm("ld.global.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
+      : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+      : "l"(p));
+  return r;
+}
+
 __device__ __forceinline__ void st_f4(float* p, float a, float b, float c, float d) {
   asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
                "f"(d)
@@ -199,6 +208,8 @@ struct RsArgs {
   int64_t head;                       // scalar elements before the first aligned group
   int64_t nvec;                       // aligned groups of 8 elements
   int32_t* device_error;              // sticky error word, or null
+  int32_t accumulate;                 // 1: R += this pass's sum (later micro-batches)
+  int32_t want_sumsq;                 // 1: accumulate the sum of squares (last pass)
 };
 
 // Pipeline shape of the reduce-scatter: each of kRsStages shared-memory stages holds the
@@ -228,6 +239,32 @@ __host__ __device__ constexpr size_t rs_smem_bytes() {
 // Each CTA writes its ss to its own slot; the finalize kernel adds the slots in a fixed
 // order. A wait that gives up (about one second) ends the CTA's pipeline early and
 // records a code in *device_error when that pointer is set.
+// The rank-ordered sums acc[0..7] of elements R[0..7]: add what earlier micro-batches
+// left in R (accumulate), store, and add the squares of the stored values to ss.
+__device__ __forceinline__ void finish8(const RsArgs& a, float* R, float (&acc)[8], double& ss) {
+  if (a.accumulate) {
+    const float4 o0 = ld_f4(R), o1 = ld_f4(R + 4);
+    acc[0] = __fadd_rn(o0.x, acc[0]);
+    acc[1] = __fadd_rn(o0.y, acc[1]);
+    acc[2] = __fadd_rn(o0.z, acc[2]);
+    acc[3] = __fadd_rn(o0.w, acc[3]);
+    acc[4] = __fadd_rn(o1.x, acc[4]);
+    acc[5] = __fadd_rn(o1.y, acc[5]);
+    acc[6] = __fadd_rn(o1.z, acc[6]);
+    acc[7] = __fadd_rn(o1.w, acc[7]);
+  }
+  // R is read back only after every bucket of the step: stream it past the caches
+  st_cs_f4(R, acc[0], acc[1], acc[2], acc[3]);
+  st_cs_f4(R + 4, acc[4], acc[5], acc[6], acc[7]);
+  if (a.want_sumsq) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const double d = (double)acc[j];
+      ss = __fma_rn(d, d, ss);
+    }
+  }
+}
+
 template <int W, int DT>
 __global__ void __launch_bounds__(kRsTmaThreads, 1)
     rs_bucket_kernel(const __grid_constant__ RsArgs a) {
@@ -293,14 +330,7 @@ __global__ void __launch_bounds__(kRsTmaThreads, 1)
 #pragma unroll
           for (int j = 0; j < 8; ++j) acc[j] = __fadd_rn(acc[j], x[j]);
         }
-        // R is read back only after every bucket of the step: stream it past the caches
-        st_cs_f4(a.R + off + e, acc[0], acc[1], acc[2], acc[3]);
-        st_cs_f4(a.R + off + e + 4, acc[4], acc[5], acc[6], acc[7]);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const double d = (double)acc[j];
-          ss = __fma_rn(d, d, ss);
-        }
+        finish8(a, a.R + off + e, acc, ss);
       }
       __syncwarp();
       if ((tid & 31) == 0) mbar_arrive(&empty[st]);
@@ -320,13 +350,7 @@ __global__ void __launch_bounds__(kRsTmaThreads, 1)
 #pragma unroll
           for (int j = 0; j < 8; ++j) acc[j] = __fadd_rn(acc[j], x[j]);
         }
-        st_cs_f4(a.R + e, acc[0], acc[1], acc[2], acc[3]);
-        st_cs_f4(a.R + e + 4, acc[4], acc[5], acc[6], acc[7]);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const double d = (double)acc[j];
-          ss = __fma_rn(d, d, ss);
-        }
+        finish8(a, a.R + e, acc, ss);
       }
       // scalar elements: the unaligned head [0, head) and the last (len - vec_end)
       const int64_t n_scalar = a.head + (a.len - vec_end);
@@ -335,9 +359,12 @@ __global__ void __launch_bounds__(kRsTmaThreads, 1)
         float acc = half_bits_to_float<DT>(a.g[0][i]);
 #pragma unroll
         for (int r = 1; r < W; ++r) acc = __fadd_rn(acc, half_bits_to_float<DT>(a.g[r][i]));
+        if (a.accumulate) acc = __fadd_rn(a.R[i], acc);
         a.R[i] = acc;
-        const double d = (double)acc;
-        ss = __fma_rn(d, d, ss);
+        if (a.want_sumsq) {
+          const double d = (double)acc;
+          ss = __fma_rn(d, d, ss);
+        }
       }
     }
   }
@@ -711,6 +738,16 @@ __global__ void state_init_kernel(WsHeader* h, zero_scaler_cfg cfg) {
   r.adam_t = 0;
 }
 
+// One thread waits on a phase of its own shared-memory barrier that nothing completes
+// (no arrivals, no copies in flight): the bounded wait gives up after about one second
+// and records code 64 in the sticky error word.
+__global__ void selftest_wait_kernel(int32_t* device_error) {
+  __shared__ uint64_t bar;
+  mbar_init(&bar, 1);
+  mbar_init_fence();
+  if (!mbar_wait(&bar, 0)) atomicOr(device_error, 64);
+}
+
 __global__ void state_write_kernel(WsHeader* h, zero_scaler_state st) {
   h->scale = st.scale;
   h->cur_hysteresis = st.cur_hysteresis;
@@ -786,6 +823,11 @@ cudaError_t launch_state_init(void* ws, const zero_scaler_cfg& cfg, cudaStream_t
   return cudaGetLastError();
 }
 
+cudaError_t launch_selftest_wait(void* ws, cudaStream_t s) {
+  selftest_wait_kernel<<<1, 1, 0, s>>>(&((WsHeader*)ws)->result.device_error);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_state_write(void* ws, const zero_scaler_state& st, cudaStream_t s) {
   state_write_kernel<<<1, 1, 0, s>>>((WsHeader*)ws, st);
   return cudaGetLastError();
@@ -793,9 +835,12 @@ cudaError_t launch_state_write(void* ws, const zero_scaler_state& st, cudaStream
 
 cudaError_t launch_reduce_scatter(int world, int dtype, const uint16_t* const* g, float* R,
                                   int64_t len, double* partial, int32_t* bucket_blocks,
-                                  int32_t* device_error, int grid, cudaStream_t s) {
+                                  int32_t* device_error, int grid, cudaStream_t s,
+                                  int accumulate, int want_sumsq) {
   RsArgs a;
   a.device_error = device_error;
+  a.accumulate = accumulate;
+  a.want_sumsq = want_sumsq;
   for (int r = 0; r < ZERO_MAX_WORLD; ++r) a.g[r] = r < world ? g[r] : nullptr;
   a.R = R;
   a.partial = partial;

@@ -66,6 +66,9 @@ struct zero_plan {
   // per-step bookkeeping (host side)
   std::vector<uint8_t> reduced;
   int64_t reduced_count = 0;
+  // gradient accumulation: next micro-batch expected per bucket, and the step's count
+  std::vector<int32_t> next_micro;
+  int32_t n_micro = 0;
   bool finalized = false;  // finalize ran and no update consumed it yet
   bool local_summed = false;  // one rank: its local sum of squares was taken this step
   size_t ws_bucket_blocks_off = 0;  // int32 per bucket: blocks of its last launch
@@ -87,9 +90,13 @@ cudaError_t rs_grid(int64_t len, int world, int dtype, int* grid);
 // Launchers (kernels.cu). All return cudaSuccess or the launch error.
 cudaError_t launch_state_init(void* ws, const zero_scaler_cfg& cfg, cudaStream_t s);
 cudaError_t launch_state_write(void* ws, const zero_scaler_state& st, cudaStream_t s);
+cudaError_t launch_selftest_wait(void* ws, cudaStream_t s);
+// accumulate: R += the pass's sum (micro-batches after the first); want_sumsq: write
+// the per-block sums of squares (the last pass of a step)
 cudaError_t launch_reduce_scatter(int world, int dtype, const uint16_t* const* g, float* R,
                                   int64_t len, double* partial, int32_t* bucket_blocks,
-                                  int32_t* device_error, int grid, cudaStream_t s);
+                                  int32_t* device_error, int grid, cudaStream_t s,
+                                  int accumulate = 0, int want_sumsq = 1);
 cudaError_t launch_finalize(void* ws, const int32_t* bucket_blocks, int64_t slots_full,
                             const double* partial, int64_t n_buckets,
                             const zero_adamw_cfg& cfg, cudaStream_t s);

@@ -141,7 +141,9 @@ class CudaRankBackend:
         zero_step_finalize_ranks(self.plan, self.adamw, s_all, self.workspace, self._s())
 
     def update(self) -> None:
-        dst = self.peer_params if self.fused_all_gather else [self.params.data_ptr()]
+        off = 2 * self.rank * self.p  # bytes to this rank's slice of a gathered buffer
+        base = self.peer_params if self.fused_all_gather else [self.params.data_ptr()]
+        dst = [q + off for q in base]
         zero_step_update_partition(self.plan, self.rank, self.master, self.exp_avg,
                                    self.exp_avg_sq, self.reduced, dst, self.dtype,
                                    self.workspace, self._s())

@@ -15,8 +15,8 @@ import torch
 
 from . import (AdamWCfg, Plan, ScalerCfg, adamw_cfg, scaler_cfg, zero_all_gather,
                zero_cast_params, zero_get_result, zero_reduce_scatter_bucket,
-               zero_reduce_scatter_bucket_host, zero_state_init, zero_step,
-               zero_step_finalize, zero_step_update)
+               zero_reduce_scatter_bucket_accum, zero_reduce_scatter_bucket_host,
+               zero_state_init, zero_step, zero_step_finalize, zero_step_update)
 
 _TORCH_HALF = {"bf16": torch.bfloat16, "fp16": torch.float16}
 
@@ -55,6 +55,13 @@ class ZeroOptimizer:
     def reduce_scatter_bucket(self, bucket: int, replica_grads: Sequence, base_offset: int = 0):
         zero_reduce_scatter_bucket(self.plan, bucket, self.dtype, replica_grads, base_offset,
                                    self.reduced, self.workspace, self._s())
+
+    def reduce_scatter_bucket_accum(self, bucket: int, micro: int, n_micro: int,
+                                    replica_grads: Sequence, base_offset: int = 0):
+        """Micro-batch `micro` of `n_micro` (gradient accumulation) for one bucket."""
+        zero_reduce_scatter_bucket_accum(self.plan, bucket, micro, n_micro, self.dtype,
+                                         replica_grads, base_offset, self.reduced,
+                                         self.workspace, self._s())
 
     def reduce_scatter_bucket_host(self, bucket: int, host_replica_grads: Sequence,
                                    host_base_offset: int, device_staging: Sequence):
