@@ -315,7 +315,7 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "bf16+fp32" if wl.gdtype == "bf16" else "fp16+fp32",
+            "dtype": "f32",  # arithmetic of the step (half inputs, fp64 norm)
             "data": "synthetic (seeded Philox gradients and init; random-init weights of the shape list)",
             "config": {
                 "workload": f"{wl.name}_w{W}",
@@ -604,7 +604,7 @@ def run_reference(args, rank: int):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16+fp32" if wl.gdtype == "bf16" else "fp16+fp32",
+        "dtype": "f32",
         "data": "synthetic (seeded Philox gradients and init)",
         "config": {"workload": f"{wl.name}_w{wl.world}", "params": wl.n, "W": wl.world,
                    "reduce_bucket_size": wl.bucket},

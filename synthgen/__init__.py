@@ -65,7 +65,6 @@ def host_lib():
         if not os.path.exists(HOST_LIB):
             build(cuda=False)
         lib = ctypes.CDLL(HOST_LIB)
-        u16p = ctypes.POINTER(ctypes.c_uint16)
         lib.synth_round_double_host.restype = ctypes.c_uint16
         lib.synth_round_double_host.argtypes = [ctypes.c_double, ctypes.c_int]
         lib.synth_round_double_array_host.argtypes = [
@@ -91,7 +90,6 @@ def host_lib():
         lib.synth_master_at_host.argtypes = [
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint32,
             ctypes.c_double]
-        del u16p
         _host = lib
     return _host
 

@@ -10,7 +10,7 @@ import synthgen
 from synthgen import device as sdev
 from zero_sharded_mixed_replica_b200 import checkpoint as ck
 
-from harness import HALF, check_all, make_opt, run_resident, stream, to_np
+from harness import HALF, check_all, run_resident, stream
 
 pytestmark = pytest.mark.gpu
 

@@ -3,7 +3,6 @@ inputs: every workload, edge shapes, overflow cases, the loss scaler, the auxili
 calls. Integer / flag state bit-exact; fp32 master, m, v within 1e-6 relative (floor:
 rms of the rank's partition); global norm within 1e-5 relative; half params within
 1 ulp; reduced gradient bit-exact."""
-import copy
 import gc
 import math
 

@@ -4,8 +4,6 @@ multi-process run are played one after another in one process and one stream (no
 kernel waits on another), each with its own plan, workspace and partition buffers; the
 update writes every rank's half values into all W gathered buffers, as the fused
 all-gather does over NVLink. Results must equal the CPU oracle's whole-model step."""
-import math
-
 import numpy as np
 import pytest
 import torch

@@ -3,7 +3,6 @@ import bisect
 import math
 
 import numpy as np
-import pytest
 
 import synthgen
 

@@ -22,7 +22,7 @@ from __future__ import annotations
 import hashlib
 import json
 import os
-from typing import Dict, Optional, Sequence, Tuple
+from typing import Optional, Sequence, Tuple
 
 import numpy as np
 

@@ -2,6 +2,7 @@
 // argument checks, host-side step bookkeeping and the launches.
 #include <cuda_runtime.h>
 #include <math.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -72,6 +73,12 @@ int reduce_bucket(zero_plan* plan, int64_t b, int32_t dt, const uint16_t* const*
   }
   return ZERO_OK;
 }
+
+// NVTX range for the lifetime of a scope (a no-op unless a profiler is attached)
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 
 int check_bucket_call(zero_plan* plan, int64_t bucket, int32_t dt, float* reduced,
                       void* ws) {
@@ -374,6 +381,7 @@ int zero_cast_params(const zero_plan* plan, const float* master, void* params,
 int zero_reduce_scatter_bucket(zero_plan* plan, int64_t bucket, int32_t grad_dtype,
                                const void* const* replica_grads, int64_t replica_base_offset,
                                float* reduced, void* workspace, void* stream) {
+  NvtxRange nvtx("zero_reduce_scatter_bucket");
   if (int rc = check_bucket_call(plan, bucket, grad_dtype, reduced, workspace)) return rc;
   if (!replica_grads) return fail(ZERO_EINVAL, "replica_grads is NULL");
   const int64_t start = bucket * plan->bucket;
@@ -449,6 +457,7 @@ int zero_reduce_scatter_bucket_accum(zero_plan* plan, int64_t bucket, int32_t mi
 
 int zero_step_finalize(zero_plan* plan, const zero_adamw_cfg* cfg, void* workspace,
                        void* stream) {
+  NvtxRange nvtx("zero_step_finalize");
   if (!plan || !workspace) return fail(ZERO_EINVAL, "NULL argument");
   if (int rc = check_adamw(cfg)) return rc;
   if (!aligned16(workspace)) return fail(ZERO_EALIGN, "workspace must be 16-byte aligned");
@@ -471,6 +480,7 @@ int zero_step_finalize(zero_plan* plan, const zero_adamw_cfg* cfg, void* workspa
 int zero_step_update(zero_plan* plan, float* master, float* exp_avg, float* exp_avg_sq,
                      const float* reduced, void* params, int32_t param_dtype,
                      const void* workspace, void* stream) {
+  NvtxRange nvtx("zero_step_update");
   if (!plan || !workspace) return fail(ZERO_EINVAL, "NULL argument");
   if (plan->n_pad > 0 && (!master || !exp_avg || !exp_avg_sq || !reduced || !params))
     return fail(ZERO_EINVAL, "NULL argument");

@@ -14,7 +14,16 @@ namespace {
 
 constexpr int kGatherThreads = 256;
 constexpr int kGatherMaxPieces = 64;
-constexpr int64_t kGatherChunk = 1 << 15;  // elements per block per piece
+constexpr int64_t kGatherChunk = 1 << 16;  // elements per block per piece
+constexpr int kGatherUnroll = 4;           // 16-byte loads in flight per thread
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
 
 struct GatherArgs {
   const uint16_t* src[kGatherMaxPieces];
@@ -40,7 +49,19 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const __grid_con
     const int64_t nvec = (hi - h) / 8;
     const uint4* vs = (const uint4*)(s + h);
     uint4* vd = (uint4*)(d + h);
-    for (int64_t v = threadIdx.x; v < nvec; v += kGatherThreads) vd[v] = vs[v];
+    for (int64_t v0 = threadIdx.x; v0 < nvec; v0 += kGatherUnroll * kGatherThreads) {
+      uint4 x[kGatherUnroll];
+#pragma unroll
+      for (int u = 0; u < kGatherUnroll; ++u) {
+        const int64_t v = v0 + (int64_t)u * kGatherThreads;
+        if (v < nvec) x[u] = ld_stream(vs + v);
+      }
+#pragma unroll
+      for (int u = 0; u < kGatherUnroll; ++u) {
+        const int64_t v = v0 + (int64_t)u * kGatherThreads;
+        if (v < nvec) vd[v] = x[u];
+      }
+    }
     for (int64_t i = h + 8 * nvec + threadIdx.x; i < hi; i += kGatherThreads) d[i] = s[i];
   } else {
     for (int64_t i = lo + threadIdx.x; i < hi; i += kGatherThreads) d[i] = s[i];
