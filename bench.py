@@ -59,6 +59,8 @@ def parse_args():
     ap.add_argument("--sweep-log2n", default="24,26,28,30")
     ap.add_argument("--sweep-world", default="1,2,4,8,16")
     ap.add_argument("--sweep-dtype", default="bf16,fp16")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay each step from a CUDA graph (launch-bound small workloads)")
     ap.add_argument("--zero3", action="store_true",
                     help="ZeRO-3 forward gather / release over the 7B tensor list")
     return ap.parse_args()
@@ -105,12 +107,13 @@ def profiled_traffic(kernel: str, workload: str):
     if not os.path.exists(path):
         return None
     src_hash, traffic = None, None
+    hash_key, traffic_key = "kernels.cu sha256[:16]:", "dram bytes per launch:"
     with open(path) as f:
         for line in f:
-            if line.startswith("kernels.cu sha256[:16]:"):
-                src_hash = line.split(":", 1)[1].strip()
-            if line.startswith("dram bytes per launch:"):
-                traffic = float(line.split(":", 1)[1].strip().split()[0])
+            if line.startswith(hash_key):
+                src_hash = line[len(hash_key):].strip()
+            if line.startswith(traffic_key):
+                traffic = float(line[len(traffic_key):].split()[0])
     if src_hash != kernel_source_hash():
         return None
     return traffic
@@ -232,6 +235,28 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
         if timed >= 0:
             ev_k3[timed][1].record(s)
 
+    graphs = None
+    if args.graph:
+        # one graph per replica slot; replays keep all step state on the device
+        graphs = []
+        for k in range(2 if wl.streaming else 1):
+            g = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(s)
+            keep = opt.stream
+            opt.stream = side
+            with torch.cuda.stream(side), torch.cuda.graph(g, stream=side):
+                for b in range(nb):
+                    opt.reduce_scatter_bucket(b, slots[k],
+                                              base_offset=b * wl.bucket if wl.streaming else 0)
+                opt.step()
+            opt.stream = keep
+            s.wait_stream(side)
+            graphs.append(g)
+
+        def one_step(t: int, timed: int = -1):  # noqa: F811  (graph replay)
+            graphs[(t - 1) % len(graphs)].replay()
+
     step_no = 0
     for _ in range(args.warmup):
         step_no += 1
@@ -279,9 +304,12 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
               "gbs": (2 + 2 * n_dst) * n_pad / (k4_ms / 1e3) / 1e9}
         del dst
 
-    k1_ms = [a.elapsed_time(b) for a, b in ev_k1]
-    k2_ms = [a.elapsed_time(b) for a, b in ev_k2]
-    k3_ms = [a.elapsed_time(b) for a, b in ev_k3]
+    if graphs is None:
+        k1_ms = [a.elapsed_time(b) for a, b in ev_k1]
+        k2_ms = [a.elapsed_time(b) for a, b in ev_k2]
+        k3_ms = [a.elapsed_time(b) for a, b in ev_k3]
+    else:  # no events inside a graph: only whole steps are timed
+        k1_ms = k2_ms = k3_ms = [float("nan")]
 
     ms_max = ms_total
     if world_size > 1:
@@ -350,11 +378,19 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
                 "algorithmic_bytes_per_launch": k3_bytes,
             },
             "gpu_launches": args.steps * (nb + 2),
+            "cuda_graph": bool(graphs),
             "clocks": clocks,
             "wall_s_timed": t_wall,
             "last_result": {k: res[k] for k in ("global_norm", "clip_coef", "adam_t", "skipped")},
         }
-    del opt, slots
+    if rank == 0 and graphs:
+        out["stage_ms"] = None
+        out["reduce_scatter_gbs"] = None
+        out["roofline"] = {"kernel": "whole step (CUDA graph replay)", "bound": "hbm",
+                           "achieved": sched_gbs, "peak": peak, "peak_kind": peak_kind,
+                           "unit": "GB/s", "frac": sched_gbs / peak, "traffic": None,
+                           "algorithmic_bytes_per_launch": schedule_bytes_per_param(W) * n_pad}
+    del opt, slots, graphs
     torch.cuda.empty_cache()
     return out
 
@@ -536,9 +572,25 @@ def run_zero3_forward(args, local_rank: int) -> dict:
     fetched = sched.stats["fetched_elements"]
     peak, kind = measured_peaks()
     gbs = 4 * fetched / (ms / 1e3) / 1e9  # 2 B read + 2 B written per gathered element
+    # the gather kernel alone, on the largest fetch of the pass
+    big = max((ids for op, _, ids in sched.events if op == zb.ZERO3_FETCH),
+              key=lambda ids: sum(plan.tensor_table[t][1] for t in ids))
+    n_big = sum(plan.tensor_table[t][1] for t in big)
+    dst = torch.empty(n_big, dtype=torch.bfloat16, device=dev)
+    zb.zero3_gather(plan, big, parts, dst, s.cuda_stream)
+    e0.record(s)
+    for _ in range(10):
+        zb.zero3_gather(plan, big, parts, dst, s.cuda_stream)
+    e1.record(s)
+    torch.cuda.synchronize(dev)
+    k_ms = e0.elapsed_time(e1) / 10
+    k_gbs = 4 * n_big / (k_ms / 1e3) / 1e9
     return {"mode": "zero3_forward_gather", "workload": "llama7b_w8", "passes": passes,
             "ms_per_forward": ms, "gathered_elements": fetched,
-            "copy_gbs": gbs, "frac_of_peak": gbs / peak, "schedule": sched.stats}
+            "copy_gbs": gbs, "frac_of_peak": gbs / peak,
+            "gather_kernel": {"elements": n_big, "tensors": len(big), "ms": k_ms,
+                              "copy_gbs": k_gbs, "frac_of_peak": k_gbs / peak},
+            "schedule": sched.stats}
 
 
 # ---------------------------------------------------------------------------- oracle arm

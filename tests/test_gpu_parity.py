@@ -460,3 +460,40 @@ def test_bounded_wait_gives_up_and_reports():
     g = [torch.zeros(opt.plan.n_pad, dtype=torch.bfloat16, device="cuda")] * 2
     opt.full_step(g)
     assert opt.result()["device_error"] == 0
+
+
+# ----------------------------------------------------------------------------- CUDA graphs
+
+def test_captured_step_replays_like_eager_steps():
+    """A CUDA graph of one step, replayed 4 times (an overflow in the replica buffers
+    before the third replay), equals 4 eager steps bit for bit, scaler state included."""
+    wl = synthgen.Workload("graph", [synthgen.TensorSpec("w", (300000,), "normal"),
+                                     synthgen.TensorSpec("b", (77,), "zeros")], world=4,
+                           bucket=100000, steps=4, gdtype="fp16", dynamic=True, grad_sigma=1e-2)
+    outs = []
+    for mode in ("eager", "graph"):
+        opt = make_opt(wl)
+        s = stream()
+        sdev.init_master(wl, opt.master, s)
+        opt.cast_params()
+        g = [torch.zeros(opt.plan.n_pad, dtype=torch.float16, device="cuda") for _ in range(4)]
+        sdev.fill_grads(wl, g, 0, wl.n, 1, 2.0 ** 16, s)
+        graph = opt.capture_step(g) if mode == "graph" else None
+        for t in range(4):
+            if t == 2:
+                g[1][123] = float("inf")
+            if t == 3:
+                g[1][123] = 0.0
+            if graph is None:
+                opt.full_step(g)
+            else:
+                graph.replay()
+        torch.cuda.synchronize()
+        outs.append((opt.result(), [to_np(x).copy() for x in (opt.master, opt.exp_avg,
+                                                               opt.exp_avg_sq, opt.params)]))
+    (re, ae), (rg, ag) = outs
+    for k in ("adam_t", "iter", "next_scale", "hysteresis", "global_norm", "skipped"):
+        assert re[k] == rg[k], k
+    assert re["adam_t"] == 3
+    for a, b in zip(ae, ag):
+        assert np.array_equal(a.view(np.uint8), b.view(np.uint8))

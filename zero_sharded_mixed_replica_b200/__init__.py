@@ -249,6 +249,13 @@ class Plan:
         _check(lib.zero_plan_tensor(self._h, t, ctypes.byref(off), ctypes.byref(num)))
         return off.value, num.value
 
+    @property
+    def tensor_table(self) -> List[tuple]:
+        """(flat offset, numel) of every tensor, read once."""
+        if getattr(self, "_table", None) is None:
+            self._table = [self.tensor(t) for t in range(self.info.n_tensors)]
+        return self._table
+
     def bucket(self, b: int):
         s, ln = ctypes.c_int64(), ctypes.c_int64()
         _check(lib.zero_plan_bucket(self._h, b, ctypes.byref(s), ctypes.byref(ln)))

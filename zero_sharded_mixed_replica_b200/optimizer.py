@@ -93,3 +93,22 @@ class ZeroOptimizer:
         for b in range(self.plan.n_buckets):
             self.reduce_scatter_bucket(b, replica_grads, base_offset)
         self.step()
+
+    def capture_step(self, replica_grads: Sequence, base_offset: int = 0) -> torch.cuda.CUDAGraph:
+        """A CUDA graph of one full step over fixed replica buffers (every launch of the
+        step, no host work): `graph.replay()` runs a step. The step allocates nothing and
+        never synchronises, so it captures as is; the loss-scaler state stays on the device,
+        so replays keep skipping, scaling and counting steps like eager calls. Capture on a
+        side stream, as CUDA graphs require; the plan's host bookkeeping sees one step."""
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        keep = self.stream
+        self.stream = side
+        try:
+            with torch.cuda.stream(side), torch.cuda.graph(graph, stream=side):
+                self.full_step(replica_grads, base_offset)
+        finally:
+            self.stream = keep
+        torch.cuda.current_stream(self.device).wait_stream(side)
+        return graph

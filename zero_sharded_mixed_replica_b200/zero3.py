@@ -26,13 +26,14 @@ def run_forward(plan: Plan, schedule: Zero3Schedule, partitions: Sequence[int],
                 device="cuda", stream=None) -> dict:
     """Executes the schedule; `on_layer(layer, {tensor id: flat view})` stands for the
     layer's forward computation. Returns live-memory statistics in elements."""
+    table = plan.tensor_table
     live: Dict[int, tuple] = {}      # tensor id -> (buffer id, offset)
     buffers: Dict[int, list] = {}    # buffer id -> [tensor, remaining tensors]
     next_id, live_elems, peak = 0, 0, 0
     s = stream if stream is not None else torch.cuda.current_stream().cuda_stream
     for op, layer, ids in schedule.events:
         if op == ZERO3_FETCH:
-            sizes = [plan.tensor(t)[1] for t in ids]
+            sizes = [table[t][1] for t in ids]
             buf = torch.empty(sum(sizes), dtype=dtype, device=device)
             zero3_gather(plan, ids, partitions, buf, s)
             off = 0
@@ -44,15 +45,12 @@ def run_forward(plan: Plan, schedule: Zero3Schedule, partitions: Sequence[int],
             live_elems += sum(sizes)
             peak = max(peak, live_elems)
         elif op == ZERO3_COMPUTE:
-            views = {}
-            for t, (b, off) in live.items():
-                n = plan.tensor(t)[1]
-                views[t] = buffers[b][0][off:off + n]
+            views = {t: buffers[b][0][off:off + table[t][1]] for t, (b, off) in live.items()}
             on_layer(layer, views)
         elif op == ZERO3_RELEASE:
             for t in ids:
                 b, _ = live.pop(t)
-                live_elems -= plan.tensor(t)[1]
+                live_elems -= table[t][1]
                 buffers[b][1] -= 1
                 if buffers[b][1] == 0:
                     del buffers[b]
