@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define ZERO_ABI_VERSION 1
+#define ZERO_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define ZERO_API __attribute__((visibility("default")))
@@ -327,13 +327,24 @@ ZERO_API int zero_step_update_partition(zero_plan* plan, int32_t rank, float* ma
                                         int32_t n_dst, int32_t param_dtype,
                                         const void* workspace, void* stream);
 
-/* Peer memory: CUDA IPC handles (ZERO_IPC_HANDLE_BYTES opaque bytes) so that rank q's
+/* Peer memory: CUDA IPC handles (zero_ipc_handle_bytes() opaque bytes) so that rank q's
  * buffers can be read and written by the other ranks' kernels over NVLink. The caller
- * moves the handle bytes between processes (e.g. an all-gather of objects). */
+ * moves the handle bytes and the offset between processes (e.g. an all-gather of
+ * objects).
+ *   zero_ipc_get_handle: a handle to the device allocation that holds device_ptr, and in
+ *       *offset_out the byte offset of device_ptr from that allocation's start (a pool
+ *       allocator such as torch's places many buffers in one allocation).
+ *   zero_ipc_open_handle: maps the peer's whole allocation into this process and returns
+ *       its start in *base_out; the peer's buffer is at base + offset. The mapping stays
+ *       valid until zero_ipc_close(base) and the exporter must keep the allocation alive
+ *       until every peer has closed it. A handle exported by this process cannot be
+ *       opened by it (use the pointer itself).
+ * Errors: EINVAL for NULL arguments; ECUDA when the runtime refuses (the message names
+ * the call). */
 ZERO_API int zero_ipc_handle_bytes(void);
-ZERO_API int zero_ipc_get_handle(const void* device_ptr, void* handle_out);
-ZERO_API int zero_ipc_open_handle(const void* handle, void** device_ptr);
-ZERO_API int zero_ipc_close(void* device_ptr);
+ZERO_API int zero_ipc_get_handle(const void* device_ptr, void* handle_out, int64_t* offset_out);
+ZERO_API int zero_ipc_open_handle(const void* handle, void** base_out);
+ZERO_API int zero_ipc_close(void* base);
 
 /* ---------------------------------------------------------------- ZeRO-3 parameters
  * Stage 3 partitions the half parameters too ([Z1] 1.2.3; [Z2]; [Z3] technical insight):

@@ -111,6 +111,9 @@ class Memory(ctypes.Structure):
                 ("optimizer_state", ctypes.c_double), ("total", ctypes.c_double)]
 
 
+ABI_VERSION = 2  # must equal ZERO_ABI_VERSION of include/zero_b200.h
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
@@ -146,7 +149,7 @@ def _load():
         "zero_step_finalize_ranks": [vp, P(AdamWCfg), vp, vp, vp],
         "zero_step_update_partition": [vp, i32, vp, vp, vp, vp, vp, i32, i32, vp, vp],
         "zero_ipc_handle_bytes": [],
-        "zero_ipc_get_handle": [vp, vp],
+        "zero_ipc_get_handle": [vp, vp, P(i64)],
         "zero_ipc_open_handle": [vp, P(vp)],
         "zero_ipc_close": [vp],
         "zero_reduce_sumsq_noalloc": [i32, i32, vp, i64, vp, vp, vp],
@@ -167,6 +170,9 @@ def _load():
     L.zero_plan_destroy.restype = None
     L.zero3_schedule_destroy.restype = None
     L.zero_last_error.restype = ctypes.c_char_p
+    if L.zero_abi_version() != ABI_VERSION:
+        raise ImportError(f"{LIB_PATH} has ABI {L.zero_abi_version()}, this binding wants "
+                          f"{ABI_VERSION}: rebuild the library")
     return L
 
 
@@ -470,21 +476,24 @@ def zero_step_update_partition(plan: Plan, rank: int, master_local, exp_avg_loca
         _addr(workspace), _stream(stream)))
 
 
-def zero_ipc_get_handle(device_ptr) -> bytes:
+def zero_ipc_get_handle(device_ptr) -> tuple:
+    """(handle bytes, byte offset of the pointer in its allocation)."""
     buf = ctypes.create_string_buffer(lib.zero_ipc_handle_bytes())
-    _check(lib.zero_ipc_get_handle(_addr(device_ptr), buf))
-    return buf.raw
+    off = ctypes.c_int64()
+    _check(lib.zero_ipc_get_handle(_addr(device_ptr), buf, ctypes.byref(off)))
+    return buf.raw, off.value
 
 
 def zero_ipc_open_handle(handle: bytes) -> int:
+    """Start of the peer's mapped allocation (add the exporter's offset)."""
     p = ctypes.c_void_p()
     _check(lib.zero_ipc_open_handle(ctypes.create_string_buffer(handle, len(handle)),
                                     ctypes.byref(p)))
     return int(p.value)
 
 
-def zero_ipc_close(device_ptr: int) -> None:
-    _check(lib.zero_ipc_close(device_ptr))
+def zero_ipc_close(base: int) -> None:
+    _check(lib.zero_ipc_close(ctypes.c_void_p(base)))
 
 
 def zero_reduce_sumsq_noalloc(world_size: int, grad_dtype, replica_grads: Sequence, n: int,

@@ -7,6 +7,7 @@
 #include <string.h>
 
 #include <new>
+#include <mutex>
 #include <string>
 
 #include "zero_b200.h"
@@ -685,8 +686,35 @@ int zero_selftest_bounded_wait(void* workspace, void* stream) {
 
 int zero_ipc_handle_bytes(void) { return (int)sizeof(cudaIpcMemHandle_t); }
 
-int zero_ipc_get_handle(const void* device_ptr, void* handle_out) {
-  if (!device_ptr || !handle_out) return fail(ZERO_EINVAL, "NULL argument");
+// The start of the allocation holding a device pointer, from the driver's
+// cuMemGetAddressRange, looked up through the runtime so that the library does not link
+// the driver library itself (it must load on machines without one).
+typedef int (*MemGetAddressRangeFn)(unsigned long long* base, size_t* size,
+                                    unsigned long long ptr);
+
+static int allocation_offset(const void* device_ptr, int64_t* offset) {
+  static std::once_flag once;
+  static MemGetAddressRangeFn fn = nullptr;
+  static cudaError_t lookup = cudaSuccess;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    lookup = cudaGetDriverEntryPoint("cuMemGetAddressRange", &f, cudaEnableDefault, &q);
+    if (lookup == cudaSuccess && q == cudaDriverEntryPointSuccess) fn = (MemGetAddressRangeFn)f;
+  });
+  if (!fn) return fail(ZERO_ECUDA, "cuMemGetAddressRange unavailable");
+  unsigned long long base = 0;
+  size_t size = 0;
+  const int r = fn(&base, &size, (unsigned long long)(uintptr_t)device_ptr);
+  if (r != 0) return fail(ZERO_ECUDA, "cuMemGetAddressRange failed (" + std::to_string(r) + ")");
+  *offset = (int64_t)((uintptr_t)device_ptr - (uintptr_t)base);
+  return ZERO_OK;
+}
+
+int zero_ipc_get_handle(const void* device_ptr, void* handle_out, int64_t* offset_out) {
+  if (!device_ptr || !handle_out || !offset_out) return fail(ZERO_EINVAL, "NULL argument");
+  int rc = allocation_offset(device_ptr, offset_out);
+  if (rc != ZERO_OK) return rc;
   cudaIpcMemHandle_t h;
   cudaError_t e = cudaIpcGetMemHandle(&h, (void*)device_ptr);
   if (e != cudaSuccess) return cuda_fail(e, "cudaIpcGetMemHandle");
@@ -694,18 +722,18 @@ int zero_ipc_get_handle(const void* device_ptr, void* handle_out) {
   return ZERO_OK;
 }
 
-int zero_ipc_open_handle(const void* handle, void** device_ptr) {
-  if (!handle || !device_ptr) return fail(ZERO_EINVAL, "NULL argument");
+int zero_ipc_open_handle(const void* handle, void** base_out) {
+  if (!handle || !base_out) return fail(ZERO_EINVAL, "NULL argument");
   cudaIpcMemHandle_t h;
   memcpy(&h, handle, sizeof h);
-  cudaError_t e = cudaIpcOpenMemHandle(device_ptr, h, cudaIpcMemLazyEnablePeerAccess);
+  cudaError_t e = cudaIpcOpenMemHandle(base_out, h, cudaIpcMemLazyEnablePeerAccess);
   if (e != cudaSuccess) return cuda_fail(e, "cudaIpcOpenMemHandle");
   return ZERO_OK;
 }
 
-int zero_ipc_close(void* device_ptr) {
-  if (!device_ptr) return fail(ZERO_EINVAL, "NULL argument");
-  cudaError_t e = cudaIpcCloseMemHandle(device_ptr);
+int zero_ipc_close(void* base) {
+  if (!base) return fail(ZERO_EINVAL, "NULL argument");
+  cudaError_t e = cudaIpcCloseMemHandle(base);
   if (e != cudaSuccess) return cuda_fail(e, "cudaIpcCloseMemHandle");
   return ZERO_OK;
 }

@@ -9,7 +9,10 @@ gathered buffer (the all-gather fused into the update) -- or, with
 `fused_all_gather=False`, into its own buffer followed by a collective all-gather.
 The only collectives are one all-gather of the W fp64 sums of squares (rank order, so
 every rank computes the same norm, clip and loss-scale decision) and the stream-ordered
-barriers that separate writers from peer readers.
+barriers that separate writers from peer readers. With `host_exchange=True` those
+exchanges go through the host instead (a device synchronize, then a CPU collective, e.g.
+gloo): slower, but no device work ever waits on another process's device work, which is
+what ranks that share one GPU need.
 
 Sources: [Z1] "ZeRO技术解析" 2.1 (parameters split into N parts, gradients
 reduce-scattered, each GPU updates its own partition, parameters gathered with
@@ -18,7 +21,7 @@ insight (each GPU keeps only its own gradient slice).
 """
 from __future__ import annotations
 
-from typing import List, Optional, Sequence
+from typing import Dict, List, Optional, Sequence
 
 import torch
 import torch.distributed as dist
@@ -75,7 +78,8 @@ class CudaRankBackend:
     def __init__(self, shapes: Sequence[Sequence[int]], reduce_bucket_size: int, dtype: str,
                  rank: int, world: int, group=None, align: int = 128,
                  scaler: Optional[ScalerCfg] = None, adamw: Optional[AdamWCfg] = None,
-                 fused_all_gather: bool = True, device: Optional[torch.device] = None):
+                 fused_all_gather: bool = True, device: Optional[torch.device] = None,
+                 host_exchange: bool = False):
         self.rank, self.world, self.dtype = rank, world, dtype
         self.device = device or torch.device("cuda", torch.cuda.current_device())
         self.plan = Plan(shapes, world, reduce_bucket_size, align)
@@ -93,37 +97,53 @@ class CudaRankBackend:
         self.scaler = scaler if scaler is not None else scaler_cfg(dynamic=(dtype == "fp16"))
         self.adamw = adamw if adamw is not None else adamw_cfg()
         self.fused_all_gather = fused_all_gather
+        self.host_exchange = host_exchange
         zero_state_init(self.plan, self.workspace, self.scaler, self._s())
-        # peers' buffers, mapped once (IPC handles travel through the process group)
+        # peers' buffers, mapped once (IPC handles travel through the process group). A
+        # handle names a whole allocation, which may hold both buffers: each distinct
+        # allocation is mapped once and the exporter's offset places the buffer in it.
         mine = (zero_ipc_get_handle(self.grads), zero_ipc_get_handle(self.params))
         handles: List = [None] * world
         dist.all_gather_object(handles, mine, group=group)
-        self._opened: List[int] = []
+        self._opened: Dict[bytes, int] = {}
+
+        def peer(h) -> int:
+            key, off = h
+            if key not in self._opened:
+                self._opened[key] = zero_ipc_open_handle(key)
+            return self._opened[key] + off
+
         self.peer_grads, self.peer_params = [], []
         for q in range(world):
             if q == rank:
                 self.peer_grads.append(self.grads.data_ptr())
                 self.peer_params.append(self.params.data_ptr())
             else:
-                g = zero_ipc_open_handle(handles[q][0])
-                p = zero_ipc_open_handle(handles[q][1])
-                self._opened += [g, p]
-                self.peer_grads.append(g)
-                self.peer_params.append(p)
+                self.peer_grads.append(peer(handles[q][0]))
+                self.peer_params.append(peer(handles[q][1]))
 
     def _s(self) -> int:
         return torch.cuda.current_stream(self.device).cuda_stream
 
     def close(self) -> None:
-        for ptr in self._opened:
-            zero_ipc_close(ptr)
-        self._opened = []
+        """Unmap the peers' allocations (every rank must be done reading and writing
+        them, and must call this before any rank frees its buffers)."""
+        for base in self._opened.values():
+            zero_ipc_close(base)
+        self._opened = {}
 
     def own_slice(self) -> torch.Tensor:
         return self.params[self.rank * self.p:(self.rank + 1) * self.p]
 
     # ---- the step
+    def _host_barrier(self, group) -> None:
+        torch.cuda.synchronize(self.device)
+        dist.barrier(group=group)
+
     def before_peer_reads(self, group) -> None:
+        if self.host_exchange:
+            self._host_barrier(group)
+            return
         # stream-ordered barrier: a rank's gradient writes precede its all-reduce, which
         # no rank completes before all have entered it
         flag = torch.zeros(1, device=self.device)
@@ -135,9 +155,11 @@ class CudaRankBackend:
 
     def local_sumsq(self) -> torch.Tensor:
         zero_step_local_sumsq(self.plan, self.rank, self.workspace, self.sumsq, self._s())
-        return self.sumsq
+        return self.sumsq.cpu() if self.host_exchange else self.sumsq
 
     def finalize(self, s_all: torch.Tensor) -> None:
+        if self.host_exchange:
+            s_all = s_all.to(self.device)
         zero_step_finalize_ranks(self.plan, self.adamw, s_all, self.workspace, self._s())
 
     def update(self) -> None:
@@ -149,6 +171,17 @@ class CudaRankBackend:
                                    self.workspace, self._s())
 
     def after_update(self, group) -> None:
+        if self.host_exchange:
+            if not self.fused_all_gather:
+                # the half slices travel as bytes (gloo has no 16-bit float types)
+                own = self.own_slice().cpu().view(torch.uint8)
+                parts = [torch.empty_like(own) for _ in range(self.world)]
+                dist.all_gather(parts, own, group=group)
+                self.params.copy_(torch.cat(parts).view(self.params.dtype).to(self.device))
+            # the peers' stores into this buffer (or the copy above) have landed, and
+            # every rank is done reading the peers' gradients
+            self._host_barrier(group)
+            return
         if self.fused_all_gather:
             # every rank's stores into the peers' gathered buffers have landed before any
             # rank uses its buffer
