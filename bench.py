@@ -61,6 +61,9 @@ def parse_args():
     ap.add_argument("--sweep-dtype", default="bf16,fp16")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step from a CUDA graph (launch-bound small workloads)")
+    ap.add_argument("--micro", type=int, default=1,
+                    help="gradient accumulation: micro-batches per step (each reduces every "
+                         "bucket; the later ones add into the reduced gradient)")
     ap.add_argument("--zero3", action="store_true",
                     help="ZeRO-3 forward gather / release over the 7B tensor list")
     return ap.parse_args()
@@ -213,18 +216,26 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
         sdev.fill_grads(wl, slots[k], 0, min(L, wl.n), k + 1, scale, sh)
     torch.cuda.synchronize(dev)
 
-    ev_k1 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps * nb)]
+    M = max(1, args.micro)
+    ev_k1 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)]
+             for _ in range(args.steps * nb * M)]
     ev_k3 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     ev_k2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
 
     def one_step(t: int, timed: int = -1):
         bufs = slots[(t - 1) % 2] if wl.streaming else slots[0]
-        for b in range(nb):
-            if timed >= 0:
-                ev_k1[timed * nb + b][0].record(s)
-            opt.reduce_scatter_bucket(b, bufs, base_offset=b * wl.bucket if wl.streaming else 0)
-            if timed >= 0:
-                ev_k1[timed * nb + b][1].record(s)
+        for k in range(M):  # micro-batches reuse the resident replica slot
+            for b in range(nb):
+                e = (timed * M + k) * nb + b
+                if timed >= 0:
+                    ev_k1[e][0].record(s)
+                base = b * wl.bucket if wl.streaming else 0
+                if M == 1:
+                    opt.reduce_scatter_bucket(b, bufs, base_offset=base)
+                else:
+                    opt.reduce_scatter_bucket_accum(b, k, M, bufs, base_offset=base)
+                if timed >= 0:
+                    ev_k1[e][1].record(s)
         if timed >= 0:
             ev_k2[timed][0].record(s)
         opt.step_finalize()
@@ -236,6 +247,8 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
             ev_k3[timed][1].record(s)
 
     graphs = None
+    if args.graph and M > 1:
+        raise SystemExit("--graph with --micro > 1 is not supported")
     if args.graph:
         # one graph per replica slot; replays keep all step state on the device
         graphs = []
@@ -326,11 +339,24 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
         k3_avg = sum(k3_ms) / len(k3_ms)
         k3_bytes = 30 * n_pad  # R, p, m, v read (16 B) + p, m, v write (12 B) + half (2 B)
         k3_gbs = k3_bytes / (k3_avg / 1e3) / 1e9
-        full_b = [k1_ms[i] for i in range(len(k1_ms)) if plan.bucket(i % nb)[1] == wl.bucket] or k1_ms
+        # first micro-batch passes (2W + 4 B/param) and accumulate passes (2W + 8)
+        first = [i for i in range(len(k1_ms)) if (i // nb) % M == 0]
+        later = [i for i in range(len(k1_ms)) if (i // nb) % M != 0]
+        full_b = [k1_ms[i] for i in first if plan.bucket(i % nb)[1] == wl.bucket] or \
+            [k1_ms[i] for i in first]
         k1_avg = sum(full_b) / len(full_b)
         k1_bytes = (2 * W + 4) * plan.bucket(0)[1]
-        sched_gbs = schedule_bytes_per_param(W) * n_pad / (ms_step / 1e3) / 1e9
-        model_gbs = model_bytes_per_param(W) * plan.n / (ms_step / 1e3) / 1e9
+        acc = None
+        if later and graphs is None:
+            acc_b = [k1_ms[i] for i in later if plan.bucket(i % nb)[1] == wl.bucket] or \
+                [k1_ms[i] for i in later]
+            acc_ms = sum(acc_b) / len(acc_b)
+            acc = {"ms_per_full_bucket": acc_ms,
+                   "gbs": (2 * W + 8) * plan.bucket(0)[1] / (acc_ms / 1e3) / 1e9,
+                   "bytes_per_param": 2 * W + 8}
+        step_bytes = (schedule_bytes_per_param(W) + (M - 1) * (2 * W + 8)) * n_pad
+        sched_gbs = step_bytes / (ms_step / 1e3) / 1e9
+        model_gbs = (model_bytes_per_param(W) + (M - 1) * 2 * W) * plan.n / (ms_step / 1e3) / 1e9
         traffic = profiled_traffic("adamw_cast", wl.name)
         out = {
             "metric": METRIC,
@@ -354,7 +380,8 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
                 "buckets": nb,
                 "grad_dtype": wl.gdtype,
                 "replica_buffers": "bucket-sized, 2 slots" if wl.streaming else "resident",
-                "l2": f"no flush: each step moves {schedule_bytes_per_param(W) * n_pad / 1e9:.0f} GB, inputs >> 126 MB L2",
+                "micro_batches": M,
+                "l2": f"no flush: each step moves {step_bytes / 1e9:.0f} GB, inputs >> 126 MB L2",
                 "parallelism": f"replicas x{world_size} (simulated dp{W} per GPU)",
             },
             "hbm_gbs_schedule": sched_gbs,
@@ -365,6 +392,7 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
                          "finalize": sum(k2_ms) / len(k2_ms),
                          "adamw_cast": k3_avg},
             "reduce_scatter_gbs": k1_bytes / (k1_avg / 1e3) / 1e9,
+            "accumulate_pass": acc,
             "all_gather_copies": k4,
             "roofline": {
                 "kernel": "adamw_cast_kernel",
@@ -377,7 +405,7 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
                 "traffic": traffic,
                 "algorithmic_bytes_per_launch": k3_bytes,
             },
-            "gpu_launches": args.steps * (nb + 2),
+            "gpu_launches": args.steps * (M * nb + 2),
             "cuda_graph": bool(graphs),
             "clocks": clocks,
             "wall_s_timed": t_wall,
@@ -701,6 +729,8 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     out = run_ours(args, rank, world_size, local_rank)
     wl = get_workload(args)
+    if args.micro > 1:  # the end-to-end and oracle legs time the one-micro-batch step
+        args.no_e2e = args.no_cpu_baseline = True
     if not args.no_e2e:
         e2e = run_e2e(args, wl, local_rank, world_size)  # every rank takes part
         if rank == 0:
