@@ -141,3 +141,37 @@ def test_step_call_errors_before_any_device_work():
     assert _code(zb.zero_all_gather, p, R, [0], "bf16") == zb.ZERO_EINVAL
     assert _code(zb.zero_all_gather, p, R, [R + 2], "bf16") == zb.ZERO_EALIGN
     zb.zero_all_gather(p, R, [], "bf16")  # n_dst = 0: nothing to do
+
+
+def _msg(fn, *a):
+    with pytest.raises(zb.ZeroError) as e:
+        fn(*a)
+    assert e.value.code == zb.ZERO_EINVAL
+    return e.value.message
+
+
+def test_binding_checks_tensor_arguments():
+    """Tensor arguments are checked (dtype, layout, host or device, length) before their
+    addresses reach the library; raw integer addresses are passed through."""
+    import torch
+    p = zb.Plan([(1000,)], 2, 512)
+    ws, R = 1 << 20, 2 << 20  # raw addresses: not checked, never dereferenced here
+    bf = [torch.zeros(p.n_pad, dtype=torch.bfloat16) for _ in range(2)]
+    assert "device memory" in _msg(zb.zero_reduce_scatter_bucket, p, 0, "bf16", bf, 0, R, ws)
+    fp = [torch.zeros(p.n_pad, dtype=torch.float16)] * 2
+    assert "where bf16" in _msg(zb.zero_reduce_scatter_bucket, p, 0, "bf16", fp, 0, R, ws)
+    strided = [torch.zeros(2 * p.n_pad, dtype=torch.bfloat16)[::2]] * 2
+    assert "contiguous" in _msg(zb.zero_reduce_scatter_bucket, p, 0, "bf16", strided, 0, R, ws)
+    f64 = torch.zeros(p.n_pad, dtype=torch.float64)
+    assert "where f32" in _msg(zb.zero_step, p, zb.adamw_cfg(), f64, R, R, R, R, "bf16", ws)
+    # the host-staging call wants host replicas that cover the bucket
+    b0, len0 = p.bucket(1)
+    short = [torch.zeros(b0 + len0 - 1, dtype=torch.int16)] * 2
+    assert "needs %d" % (b0 + len0) in _msg(zb.zero_reduce_scatter_bucket_host, p, 1, "bf16",
+                                             short, 0, [3 << 20, 4 << 20], R, ws)
+    # a replica buffer indexed from the bucket start needs only the bucket's length
+    based = [torch.zeros(len0 - 1, dtype=torch.int16)] * 2
+    assert "needs %d" % len0 in _msg(zb.zero_reduce_scatter_bucket_host, p, 1, "bf16", based,
+                                      b0, [3 << 20, 4 << 20], R, ws)
+    ws_host = torch.zeros(p.workspace_bytes(), dtype=torch.uint8)
+    assert "device memory" in _msg(zb.zero_state_init, p, ws_host, zb.scaler_cfg(False))

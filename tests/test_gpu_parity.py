@@ -497,3 +497,16 @@ def test_captured_step_replays_like_eager_steps():
     assert re["adam_t"] == 3
     for a, b in zip(ae, ag):
         assert np.array_equal(a.view(np.uint8), b.view(np.uint8))
+
+
+def test_binding_refuses_short_device_buffers():
+    p = zb.Plan([(5000,)], 2, 3000)
+    ws = torch.zeros(p.workspace_bytes(), dtype=torch.uint8, device="cuda")
+    g = [torch.zeros(p.n_pad, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    R = torch.zeros(p.n_pad, device="cuda")
+    for args in ((g, R[:-1], ws), (g, R, ws[:-1]), ([g[0], g[1][:p.bucket(0)[1] - 1]], R, ws)):
+        with pytest.raises(zb.ZeroError) as e:
+            zb.zero_reduce_scatter_bucket(p, 0, "bf16", args[0], 0, args[1], args[2])
+        assert e.value.code == zb.ZERO_EINVAL and "needs" in e.value.message
+    zb.zero_state_init(p, ws, zb.scaler_cfg(False))
+    zb.zero_reduce_scatter_bucket(p, 0, "bf16", g, 0, R, ws)  # the full-size call goes through

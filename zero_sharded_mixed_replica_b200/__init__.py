@@ -205,6 +205,55 @@ def _ptr_array(ptrs: Sequence) -> ctypes.Array:
     return (ctypes.c_void_p * len(ptrs))(*[_addr(p) for p in ptrs])
 
 
+# Tensor arguments are checked before their addresses cross the ABI (the library trusts
+# the lengths the plan implies, and a short buffer would be read or written out of
+# bounds on the device). Plain integers are raw addresses and are not checked.
+_HALF_DTYPES = {"bf16": ("torch.bfloat16", "torch.int16", "torch.uint16"),
+                "fp16": ("torch.float16", "torch.int16", "torch.uint16")}
+_KIND_DTYPES = {"f32": ("torch.float32",), "f64": ("torch.float64",)}
+
+
+def _buf(x, kind: str, need: int, name: str, host: bool = False) -> Optional[int]:
+    """Address of `x` after checking a tensor argument: `kind` is "f32", "f64", "bf16",
+    "fp16" or "bytes"; `need` the elements (bytes for "bytes") it must hold."""
+    if x is None or isinstance(x, int):
+        return x
+    dt = str(x.dtype)
+    if kind in _HALF_DTYPES:
+        ok, unit = dt in _HALF_DTYPES[kind], 2
+    elif kind in _KIND_DTYPES:
+        ok, unit = dt in _KIND_DTYPES[kind], 1
+    else:
+        ok, unit = True, 1
+    if not ok:
+        raise ZeroError(ZERO_EINVAL, f"{name}: dtype {dt} where {kind} is expected")
+    if not x.is_contiguous():
+        raise ZeroError(ZERO_EINVAL, f"{name}: not contiguous")
+    where = x.device.type
+    if (where == "cpu") != host:
+        raise ZeroError(ZERO_EINVAL, f"{name}: a {where} tensor where "
+                                     f"{'host' if host else 'device'} memory is expected")
+    have = x.numel() * x.element_size() if kind == "bytes" else \
+        x.numel() * x.element_size() // (2 if unit == 2 else x.element_size())
+    if have < need:
+        raise ZeroError(ZERO_EINVAL, f"{name}: holds {have} {'bytes' if kind == 'bytes' else 'elements'}"
+                                     f", needs {need}")
+    return x.data_ptr()
+
+
+def _dtype_name(dt) -> str:
+    return dt if isinstance(dt, str) else {v: k for k, v in DTYPES.items()}.get(int(dt), "?")
+
+
+def _replicas(plan, bucket: int, base: int, grads: Sequence, gdt, name: str, host=False):
+    """The replica pointer array of one bucket, each tensor checked to cover it."""
+    start, length = plan.bucket(bucket) if 0 <= bucket < plan.n_buckets else (base, 0)
+    need = max(0, start + length - int(base))
+    kind = _dtype_name(gdt)
+    return (ctypes.c_void_p * len(grads))(
+        *[_buf(g, kind, need, f"{name}[{r}]", host) for r, g in enumerate(grads)])
+
+
 def _dtype(dt) -> int:
     return DTYPES[dt] if isinstance(dt, str) else int(dt)
 
@@ -263,9 +312,13 @@ class Plan:
         return self._table
 
     def bucket(self, b: int):
-        s, ln = ctypes.c_int64(), ctypes.c_int64()
-        _check(lib.zero_plan_bucket(self._h, b, ctypes.byref(s), ctypes.byref(ln)))
-        return s.value, ln.value
+        """(start, length) of bucket b (asked of the library once per bucket)."""
+        cache = self.__dict__.setdefault("_buckets", {})
+        if b not in cache:
+            s, ln = ctypes.c_int64(), ctypes.c_int64()
+            _check(lib.zero_plan_bucket(self._h, b, ctypes.byref(s), ctypes.byref(ln)))
+            cache[b] = (s.value, ln.value)
+        return cache[b]
 
     def work_segments(self) -> List[tuple]:
         cnt = ctypes.c_int64()
@@ -287,9 +340,11 @@ class Plan:
         return {f: getattr(m, f) for f, _ in Memory._fields_}
 
     def workspace_bytes(self) -> int:
-        b = ctypes.c_size_t()
-        _check(lib.zero_workspace_bytes(self._h, ctypes.byref(b)))
-        return b.value
+        if getattr(self, "_ws_bytes", None) is None:
+            b = ctypes.c_size_t()
+            _check(lib.zero_workspace_bytes(self._h, ctypes.byref(b)))
+            self._ws_bytes = b.value
+        return self._ws_bytes
 
 
 def zero_plan_create(shapes, world_size, reduce_bucket_size, align=128) -> Plan:
@@ -315,7 +370,8 @@ def adamw_cfg(lr=6e-5, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01,
 # ---------------------------------------------------------------------------- the step
 
 def zero_state_init(plan: Plan, workspace, cfg: ScalerCfg, stream=None) -> None:
-    _check(lib.zero_state_init(plan.handle, _addr(workspace), ctypes.byref(cfg), _stream(stream)))
+    ws = _buf(workspace, "bytes", plan.workspace_bytes(), "workspace")
+    _check(lib.zero_state_init(plan.handle, ws, ctypes.byref(cfg), _stream(stream)))
 
 
 def zero_state_read(workspace, stream=None) -> dict:
@@ -326,30 +382,40 @@ def zero_state_read(workspace, stream=None) -> dict:
 
 def zero_state_write(plan: Plan, workspace, cfg: ScalerCfg, state: dict, stream=None) -> None:
     st = ScalerState(**{k: state[k] for k, _ in ScalerState._fields_})
-    _check(lib.zero_state_write(plan.handle, _addr(workspace), ctypes.byref(cfg),
+    _check(lib.zero_state_write(plan.handle, _buf(workspace, "bytes", plan.workspace_bytes(),
+                                                  "workspace"), ctypes.byref(cfg),
                                 ctypes.byref(st), _stream(stream)))
 
 
 def zero_cast_params(plan: Plan, master, params, param_dtype, stream=None) -> None:
-    _check(lib.zero_cast_params(plan.handle, _addr(master), _addr(params), _dtype(param_dtype),
-                                _stream(stream)))
+    _check(lib.zero_cast_params(plan.handle, _buf(master, "f32", plan.n_pad, "master"),
+                                _buf(params, _dtype_name(param_dtype), plan.n_pad, "params"),
+                                _dtype(param_dtype), _stream(stream)))
 
 
 def zero_reduce_scatter_bucket(plan: Plan, bucket: int, grad_dtype, replica_grads: Sequence,
                                replica_base_offset: int, reduced, workspace, stream=None) -> None:
-    _check(lib.zero_reduce_scatter_bucket(plan.handle, bucket, _dtype(grad_dtype),
-                                          _ptr_array(replica_grads), int(replica_base_offset),
-                                          _addr(reduced), _addr(workspace), _stream(stream)))
+    _check(lib.zero_reduce_scatter_bucket(
+        plan.handle, bucket, _dtype(grad_dtype),
+        _replicas(plan, bucket, replica_base_offset, replica_grads, grad_dtype, "replica_grads"),
+        int(replica_base_offset), _buf(reduced, "f32", plan.n_pad, "reduced"),
+        _buf(workspace, "bytes", plan.workspace_bytes(), "workspace"), _stream(stream)))
 
 
 def zero_reduce_scatter_bucket_host(plan: Plan, bucket: int, grad_dtype,
                                     host_replica_grads: Sequence, host_base_offset: int,
                                     device_staging: Sequence, reduced, workspace,
                                     stream=None) -> None:
+    length = plan.bucket(bucket)[1] if 0 <= bucket < plan.n_buckets else 0
+    kind = _dtype_name(grad_dtype)
+    staging = (ctypes.c_void_p * len(device_staging))(
+        *[_buf(b, kind, length, f"device_staging[{r}]") for r, b in enumerate(device_staging)])
     _check(lib.zero_reduce_scatter_bucket_host(
-        plan.handle, bucket, _dtype(grad_dtype), _ptr_array(host_replica_grads),
-        int(host_base_offset), _ptr_array(device_staging), _addr(reduced), _addr(workspace),
-        _stream(stream)))
+        plan.handle, bucket, _dtype(grad_dtype),
+        _replicas(plan, bucket, host_base_offset, host_replica_grads, grad_dtype,
+                  "host_replica_grads", host=True),
+        int(host_base_offset), staging, _buf(reduced, "f32", plan.n_pad, "reduced"),
+        _buf(workspace, "bytes", plan.workspace_bytes(), "workspace"), _stream(stream)))
 
 
 def zero_reduce_scatter_bucket_accum(plan: Plan, bucket: int, micro: int, n_micro: int,
@@ -357,33 +423,49 @@ def zero_reduce_scatter_bucket_accum(plan: Plan, bucket: int, micro: int, n_micr
                                      replica_base_offset: int, reduced, workspace,
                                      stream=None) -> None:
     _check(lib.zero_reduce_scatter_bucket_accum(
-        plan.handle, bucket, micro, n_micro, _dtype(grad_dtype), _ptr_array(replica_grads),
-        int(replica_base_offset), _addr(reduced), _addr(workspace), _stream(stream)))
+        plan.handle, bucket, micro, n_micro, _dtype(grad_dtype),
+        _replicas(plan, bucket, replica_base_offset, replica_grads, grad_dtype, "replica_grads"),
+        int(replica_base_offset), _buf(reduced, "f32", plan.n_pad, "reduced"),
+        _buf(workspace, "bytes", plan.workspace_bytes(), "workspace"), _stream(stream)))
 
 
 def zero_step(plan: Plan, cfg: AdamWCfg, master, exp_avg, exp_avg_sq, reduced, params,
               param_dtype, workspace, stream=None) -> None:
-    _check(lib.zero_step(plan.handle, ctypes.byref(cfg), _addr(master), _addr(exp_avg),
-                         _addr(exp_avg_sq), _addr(reduced), _addr(params), _dtype(param_dtype),
-                         _addr(workspace), _stream(stream)))
+    n = plan.n_pad
+    _check(lib.zero_step(plan.handle, ctypes.byref(cfg), _buf(master, "f32", n, "master"),
+                         _buf(exp_avg, "f32", n, "exp_avg"), _buf(exp_avg_sq, "f32", n, "exp_avg_sq"),
+                         _buf(reduced, "f32", n, "reduced"),
+                         _buf(params, _dtype_name(param_dtype), n, "params"), _dtype(param_dtype),
+                         _buf(workspace, "bytes", plan.workspace_bytes(), "workspace"),
+                         _stream(stream)))
 
 
 def zero_step_finalize(plan: Plan, cfg: AdamWCfg, workspace, stream=None) -> None:
-    _check(lib.zero_step_finalize(plan.handle, ctypes.byref(cfg), _addr(workspace),
+    _check(lib.zero_step_finalize(plan.handle, ctypes.byref(cfg),
+                                  _buf(workspace, "bytes", plan.workspace_bytes(), "workspace"),
                                   _stream(stream)))
 
 
 def zero_step_update(plan: Plan, master, exp_avg, exp_avg_sq, reduced, params, param_dtype,
                      workspace, stream=None) -> None:
-    _check(lib.zero_step_update(plan.handle, _addr(master), _addr(exp_avg), _addr(exp_avg_sq),
-                                _addr(reduced), _addr(params), _dtype(param_dtype),
-                                _addr(workspace), _stream(stream)))
+    n = plan.n_pad
+    _check(lib.zero_step_update(plan.handle, _buf(master, "f32", n, "master"),
+                                _buf(exp_avg, "f32", n, "exp_avg"),
+                                _buf(exp_avg_sq, "f32", n, "exp_avg_sq"),
+                                _buf(reduced, "f32", n, "reduced"),
+                                _buf(params, _dtype_name(param_dtype), n, "params"),
+                                _dtype(param_dtype),
+                                _buf(workspace, "bytes", plan.workspace_bytes(), "workspace"),
+                                _stream(stream)))
 
 
 def zero_all_gather(plan: Plan, params, rank_params: Sequence, param_dtype, stream=None) -> None:
-    arr = _ptr_array(rank_params) if rank_params else None
-    _check(lib.zero_all_gather(plan.handle, _addr(params), arr, len(rank_params),
-                               _dtype(param_dtype), _stream(stream)))
+    kind, n = _dtype_name(param_dtype), plan.n_pad
+    arr = (ctypes.c_void_p * len(rank_params))(
+        *[_buf(d, kind, n, f"rank_params[{r}]") for r, d in enumerate(rank_params)]) \
+        if rank_params else None
+    _check(lib.zero_all_gather(plan.handle, _buf(params, kind, n, "params"), arr,
+                               len(rank_params), _dtype(param_dtype), _stream(stream)))
 
 
 def zero_get_result(workspace, stream=None) -> dict:
@@ -450,30 +532,40 @@ def zero_abi_version() -> int:
 def zero_reduce_scatter_segment(plan: Plan, bucket: int, rank: int, grad_dtype,
                                 replica_grads: Sequence, replica_base_offset: int,
                                 reduced_local, workspace, stream=None) -> None:
-    _check(lib.zero_reduce_scatter_segment(plan.handle, bucket, rank, _dtype(grad_dtype),
-                                           _ptr_array(replica_grads), int(replica_base_offset),
-                                           _addr(reduced_local), _addr(workspace),
-                                           _stream(stream)))
+    _check(lib.zero_reduce_scatter_segment(
+        plan.handle, bucket, rank, _dtype(grad_dtype),
+        _replicas(plan, bucket, replica_base_offset, replica_grads, grad_dtype, "replica_grads"),
+        int(replica_base_offset), _buf(reduced_local, "f32", plan.p, "reduced_local"),
+        _buf(workspace, "bytes", plan.workspace_bytes(), "workspace"), _stream(stream)))
 
 
 def zero_step_local_sumsq(plan: Plan, rank: int, workspace, sumsq_out, stream=None) -> None:
-    _check(lib.zero_step_local_sumsq(plan.handle, rank, _addr(workspace), _addr(sumsq_out),
-                                     _stream(stream)))
+    _check(lib.zero_step_local_sumsq(plan.handle, rank,
+                                     _buf(workspace, "bytes", plan.workspace_bytes(), "workspace"),
+                                     _buf(sumsq_out, "f64", 1, "sumsq_out"), _stream(stream)))
 
 
 def zero_step_finalize_ranks(plan: Plan, cfg: AdamWCfg, sumsq_ranks, workspace,
                              stream=None) -> None:
-    _check(lib.zero_step_finalize_ranks(plan.handle, ctypes.byref(cfg), _addr(sumsq_ranks),
-                                        _addr(workspace), _stream(stream)))
+    _check(lib.zero_step_finalize_ranks(plan.handle, ctypes.byref(cfg),
+                                        _buf(sumsq_ranks, "f64", plan.world_size, "sumsq_ranks"),
+                                        _buf(workspace, "bytes", plan.workspace_bytes(),
+                                             "workspace"), _stream(stream)))
 
 
 def zero_step_update_partition(plan: Plan, rank: int, master_local, exp_avg_local,
                                exp_avg_sq_local, reduced_local, params_dst: Sequence,
                                param_dtype, workspace, stream=None) -> None:
+    p, kind = plan.p, _dtype_name(param_dtype)
+    dst = (ctypes.c_void_p * len(params_dst))(
+        *[_buf(d, kind, p, f"params_dst[{i}]") for i, d in enumerate(params_dst)])
     _check(lib.zero_step_update_partition(
-        plan.handle, rank, _addr(master_local), _addr(exp_avg_local), _addr(exp_avg_sq_local),
-        _addr(reduced_local), _ptr_array(params_dst), len(params_dst), _dtype(param_dtype),
-        _addr(workspace), _stream(stream)))
+        plan.handle, rank, _buf(master_local, "f32", p, "master_local"),
+        _buf(exp_avg_local, "f32", p, "exp_avg_local"),
+        _buf(exp_avg_sq_local, "f32", p, "exp_avg_sq_local"),
+        _buf(reduced_local, "f32", p, "reduced_local"), dst, len(params_dst),
+        _dtype(param_dtype), _buf(workspace, "bytes", plan.workspace_bytes(), "workspace"),
+        _stream(stream)))
 
 
 def zero_ipc_get_handle(device_ptr) -> tuple:

@@ -79,6 +79,17 @@ __device__ __forceinline__ void mbar_init_fence() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+// Programmatic dependent launch. The step kernels are launched with programmatic stream
+// serialization: one may be scheduled while its predecessor in the stream is finishing,
+// so each sets up its shared memory, lets its own successor be scheduled, and then waits
+// (griddepcontrol.wait: every prerequisite grid has completed and its writes are visible)
+// before it reads or writes any global memory. Without a programmatic predecessor the
+// wait returns at once.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // arrive and announce `bytes` of bulk copies that will complete on this barrier phase
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
@@ -283,6 +294,8 @@ __global__ void __launch_bounds__(kRsTmaThreads, 1)
     mbar_init_fence();
   }
   __syncthreads();
+  pdl_launch_dependents();
+  pdl_wait();
 
   const int64_t n_tiles = (8 * a.nvec) / TILE;
   const int64_t G = gridDim.x;
@@ -497,6 +510,8 @@ __device__ double sum_bucket_slots(const int32_t* __restrict__ bucket_blocks, in
 __global__ void __launch_bounds__(kFinalizeThreads)
     finalize_kernel(WsHeader* h, const int32_t* __restrict__ bucket_blocks, int64_t slots_full,
                     const double* __restrict__ partial, int64_t n_buckets, zero_adamw_cfg cfg) {
+  pdl_launch_dependents();
+  pdl_wait();
   const double S = sum_bucket_slots(bucket_blocks, slots_full, partial, 0, n_buckets);
   if (threadIdx.x == 0) finalize_scalars(h, S, cfg);
 }
@@ -566,20 +581,6 @@ constexpr size_t kUpSmemBytes = kUpStages * kUpStageBytes + 2 * kUpStages * size
 template <int DT>
 __global__ void __launch_bounds__(kUpTmaThreads, 1)
     adamw_cast_kernel(const __grid_constant__ UpArgs a) {
-  const WsHeader* h = a.h;
-  if (h->skip) return;  // overflow: the whole step is skipped
-  AdamConsts c;
-  c.k = h->k;
-  c.b1 = h->b1;
-  c.omb1 = h->omb1;
-  c.b2 = h->b2;
-  c.omb2 = h->omb2;
-  c.bc1 = h->bc1;
-  c.bc2 = h->bc2;
-  c.eps = h->eps;
-  c.lr = h->lr;
-  c.decay = h->decay;
-
   extern __shared__ __align__(128) unsigned char smem[];
   float* stage_buf = (float*)smem;  // [kUpStages][R, p, m, v][kUpTile]
   uint64_t* full = (uint64_t*)(smem + kUpStages * kUpStageBytes);
@@ -593,6 +594,22 @@ __global__ void __launch_bounds__(kUpTmaThreads, 1)
     mbar_init_fence();
   }
   __syncthreads();
+  pdl_launch_dependents();
+  pdl_wait();
+
+  const WsHeader* h = a.h;
+  if (h->skip) return;  // overflow: the whole step is skipped (every thread)
+  AdamConsts c;
+  c.k = h->k;
+  c.b1 = h->b1;
+  c.omb1 = h->omb1;
+  c.b2 = h->b2;
+  c.omb2 = h->omb2;
+  c.bc1 = h->bc1;
+  c.bc2 = h->bc2;
+  c.eps = h->eps;
+  c.lr = h->lr;
+  c.decay = h->decay;
 
   const int64_t n_tiles = a.n / kUpTile;
   const int64_t G = gridDim.x;
@@ -793,6 +810,27 @@ cudaError_t persistent_grid(const void* kernel, int threads, int64_t work_items,
 
 // ================================================================== launchers
 
+namespace {
+
+// A launch that may overlap the tail of the previous kernel in the stream (the kernel
+// waits for it before touching global memory; see pdl_wait).
+cudaError_t launch_chained(const void* kernel, dim3 grid, dim3 block, void** args,
+                           size_t smem, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, kernel, args);
+}
+
+}  // namespace
+
 int64_t rs_slots(int64_t len) {
   int64_t groups = (len + 7) / 8;
   int64_t blocks = (groups + kRsThreads - 1) / kRsThreads;
@@ -880,15 +918,16 @@ cudaError_t launch_reduce_scatter(int world, int dtype, const uint16_t* const* g
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   void* args[] = {&a};
-  return cudaLaunchKernel(k, dim3(grid), dim3(kRsTmaThreads), args, smem, s);
+  return launch_chained(k, dim3(grid), dim3(kRsTmaThreads), args, smem, s);
 }
 
 cudaError_t launch_finalize(void* ws, const int32_t* bucket_blocks, int64_t slots_full,
                             const double* partial, int64_t n_buckets,
                             const zero_adamw_cfg& cfg, cudaStream_t s) {
-  finalize_kernel<<<1, kFinalizeThreads, 0, s>>>((WsHeader*)ws, bucket_blocks, slots_full,
-                                                 partial, n_buckets, cfg);
-  return cudaGetLastError();
+  WsHeader* h = (WsHeader*)ws;
+  void* args[] = {(void*)&h, (void*)&bucket_blocks, (void*)&slots_full, (void*)&partial,
+                  (void*)&n_buckets, (void*)&cfg};
+  return launch_chained((const void*)finalize_kernel, dim3(1), dim3(kFinalizeThreads), args, 0, s);
 }
 
 cudaError_t launch_local_sumsq(const int32_t* bucket_blocks, int64_t slots_full,
@@ -935,7 +974,7 @@ cudaError_t launch_update(int dtype, const float* R, float* master, float* m, fl
   if (grid > n_tiles) grid = n_tiles;
   if (grid < 1) grid = 1;
   void* args[] = {&a};
-  return cudaLaunchKernel(k, dim3((unsigned)grid), dim3(kUpTmaThreads), args, kUpSmemBytes, s);
+  return launch_chained(k, dim3((unsigned)grid), dim3(kUpTmaThreads), args, kUpSmemBytes, s);
 }
 
 cudaError_t launch_cast(int dtype, const float* master, void* params, int64_t n,

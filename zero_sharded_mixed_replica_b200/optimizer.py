@@ -41,7 +41,17 @@ class ZeroOptimizer:
                                      device=self.device)
         self.scaler = scaler if scaler is not None else scaler_cfg(dynamic=(dtype == "fp16"))
         self.adamw = adamw if adamw is not None else adamw_cfg()
+        # the buffers allocated here are passed by address (the binding checks tensor
+        # arguments, which costs host time on small steps); one that a caller has
+        # replaced is passed as a tensor and checked
+        self._own = {k: (getattr(self, k), getattr(self, k).data_ptr()) for k in
+                     ("master", "exp_avg", "exp_avg_sq", "reduced", "params", "workspace")}
         zero_state_init(self.plan, self.workspace, self.scaler, self._s())
+
+    def _b(self, name: str):
+        t = getattr(self, name)
+        own = self._own[name]
+        return own[1] if own[0] is t else t
 
     def _s(self):
         return self.stream.cuda_stream if self.stream is not None else \
@@ -50,42 +60,44 @@ class ZeroOptimizer:
     # -------------------------------------------------------------- step pieces
     def cast_params(self) -> None:
         """params <- round_to_nearest_even(master): after initialising or loading master."""
-        zero_cast_params(self.plan, self.master, self.params, self.dtype, self._s())
+        zero_cast_params(self.plan, self._b("master"), self._b("params"), self.dtype, self._s())
 
     def reduce_scatter_bucket(self, bucket: int, replica_grads: Sequence, base_offset: int = 0):
         zero_reduce_scatter_bucket(self.plan, bucket, self.dtype, replica_grads, base_offset,
-                                   self.reduced, self.workspace, self._s())
+                                   self._b("reduced"), self._b("workspace"), self._s())
 
     def reduce_scatter_bucket_accum(self, bucket: int, micro: int, n_micro: int,
                                     replica_grads: Sequence, base_offset: int = 0):
         """Micro-batch `micro` of `n_micro` (gradient accumulation) for one bucket."""
         zero_reduce_scatter_bucket_accum(self.plan, bucket, micro, n_micro, self.dtype,
-                                         replica_grads, base_offset, self.reduced,
-                                         self.workspace, self._s())
+                                         replica_grads, base_offset, self._b("reduced"),
+                                         self._b("workspace"), self._s())
 
     def reduce_scatter_bucket_host(self, bucket: int, host_replica_grads: Sequence,
                                    host_base_offset: int, device_staging: Sequence):
         zero_reduce_scatter_bucket_host(self.plan, bucket, self.dtype, host_replica_grads,
-                                        host_base_offset, device_staging, self.reduced,
-                                        self.workspace, self._s())
+                                        host_base_offset, device_staging, self._b("reduced"),
+                                        self._b("workspace"), self._s())
 
     def step(self) -> None:
-        zero_step(self.plan, self.adamw, self.master, self.exp_avg, self.exp_avg_sq,
-                  self.reduced, self.params, self.dtype, self.workspace, self._s())
+        zero_step(self.plan, self.adamw, self._b("master"), self._b("exp_avg"),
+                  self._b("exp_avg_sq"), self._b("reduced"), self._b("params"), self.dtype,
+                  self._b("workspace"), self._s())
 
     def step_finalize(self) -> None:
-        zero_step_finalize(self.plan, self.adamw, self.workspace, self._s())
+        zero_step_finalize(self.plan, self.adamw, self._b("workspace"), self._s())
 
     def step_update(self) -> None:
-        zero_step_update(self.plan, self.master, self.exp_avg, self.exp_avg_sq, self.reduced,
-                         self.params, self.dtype, self.workspace, self._s())
+        zero_step_update(self.plan, self._b("master"), self._b("exp_avg"),
+                         self._b("exp_avg_sq"), self._b("reduced"), self._b("params"),
+                         self.dtype, self._b("workspace"), self._s())
 
     def all_gather(self, rank_params: Sequence = ()) -> None:
-        zero_all_gather(self.plan, self.params, list(rank_params), self.dtype, self._s())
+        zero_all_gather(self.plan, self._b("params"), list(rank_params), self.dtype, self._s())
 
     def result(self) -> dict:
         """Step result; synchronises the stream."""
-        return zero_get_result(self.workspace, self._s())
+        return zero_get_result(self._b("workspace"), self._s())
 
     # -------------------------------------------------------------- whole step
     def full_step(self, replica_grads: Sequence, base_offset: int = 0) -> None:
