@@ -2,6 +2,7 @@
 binding) and compares its outputs with the CPU oracle."""
 from __future__ import annotations
 
+import os
 from typing import Callable, Optional
 
 import numpy as np
@@ -94,9 +95,38 @@ def half_ulp_distance(a: np.ndarray, b: np.ndarray) -> np.ndarray:
     return np.abs(ordered(a) - ordered(b))
 
 
+# Per test and array: the fraction of bit-identical elements and the largest plain
+# relative error |got - want| / |want| (over want != 0), written out at the end of the
+# session when ZERO_PARITY_REPORT names a file (see conftest.py).
+REPORT: dict = {}
+
+
+def record(name: str, got: np.ndarray, want: np.ndarray, ulp: Optional[np.ndarray] = None):
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    entry = {"elements": int(want.size)}
+    if ulp is not None:
+        entry["identical"] = float(np.mean(ulp == 0)) if ulp.size else 1.0
+        entry["max_ulp"] = int(ulp.max()) if ulp.size else 0
+    else:
+        same = got.view(np.uint32) == want.view(np.uint32) \
+            if got.dtype == want.dtype == np.float32 else got == want
+        entry["identical"] = float(np.mean(same)) if want.size else 1.0
+        w = want.astype(np.float64)
+        nz = w != 0
+        rel = np.abs(got.astype(np.float64)[nz] - w[nz]) / np.abs(w[nz])
+        entry["max_rel"] = float(rel.max()) if rel.size else 0.0
+    cases = REPORT.setdefault(test, {})
+    key, i = name, 1
+    while key in cases:  # the same array checked again later in the test
+        i += 1
+        key = f"{name}#{i}"
+    cases[key] = entry
+
+
 def check_state(name: str, got: np.ndarray, want: np.ndarray, world: int) -> float:
     """fp32 state criterion: |got - want| <= 1e-6 * max(|want|, rms of want over the
     rank's partition). Returns the fraction of bit-identical elements."""
+    record(name, got, want)
     assert got.shape == want.shape
     n = want.size
     p = n // world if world and n % world == 0 else n
@@ -125,12 +155,14 @@ def check_scalars(res: dict, sc: dict, exact_k: bool = False) -> None:
 def check_all(opt: zb.ZeroOptimizer, ref: dict, world: int) -> dict:
     """R bit-exact, fp32 state within tolerance, params within 1 ulp."""
     R = to_np(opt.reduced)
+    record("R", R, ref["R"])
     assert np.array_equal(R.view(np.uint32), ref["R"].view(np.uint32)), \
         f"reduced gradient: {np.sum(R.view(np.uint32) != ref['R'].view(np.uint32))} elements differ"
     same = {}
     for name, t in (("master", opt.master), ("m", opt.exp_avg), ("v", opt.exp_avg_sq)):
         same[name] = check_state(name, to_np(t), ref[name], world)
     d = half_ulp_distance(to_np(opt.params), ref["params"])
+    record("params", None, ref["params"], ulp=d)
     assert d.max(initial=0) <= 1, f"params: max ulp distance {d.max()}"
     same["params"] = float(np.mean(d == 0)) if d.size else 1.0
     return same

@@ -15,7 +15,7 @@ import synthgen
 from synthgen import device as sdev
 import zero_sharded_mixed_replica_b200 as zb
 
-from harness import (HALF, check_all, check_scalars, check_state, half_ulp_distance,
+from harness import (HALF, check_all, check_scalars, check_state, half_ulp_distance, record,
                      make_opt, run_resident, run_streaming, stream, to_np)
 
 pytestmark = pytest.mark.gpu
@@ -119,14 +119,17 @@ def test_llama7b_w8_streaming_full_size_sampled():
     want = oracle.streaming_samples(wl, idx, scalars)
     it = torch.from_numpy(idx).cuda()
     got_R = opt.reduced[it].cpu().numpy()
+    record("R (sampled)", got_R, want["R"])
     assert np.array_equal(got_R.view(np.uint32), want["R"].view(np.uint32))
     for name, t in (("master", opt.master), ("m", opt.exp_avg), ("v", opt.exp_avg_sq)):
         g = t[it].cpu().numpy()
+        record(name + " (sampled)", g, want[name])
         w = want[name].astype(np.float64)
         floor = np.sqrt(np.mean(w ** 2))
         err = np.abs(g - w) / np.maximum(np.abs(w), floor)
         assert err.max() <= 1e-6, (name, err.max())
     d = half_ulp_distance(to_np(opt.params[it]), want["params"])
+    record("params (sampled)", None, want["params"], ulp=d)
     assert d.max() <= 1
     # the padding-free 7B list: invariants over the whole buffer
     assert torch.isfinite(opt.master).all().item()
