@@ -64,6 +64,10 @@ def parse_args():
     ap.add_argument("--micro", type=int, default=1,
                     help="gradient accumulation: micro-batches per step (each reduces every "
                          "bucket; the later ones add into the reduced gradient)")
+    ap.add_argument("--checkpoint", action="store_true",
+                    help="sharded checkpoint save / load (and a resharded load) of the "
+                         "optimizer state after one step; workload --checkpoint-workload")
+    ap.add_argument("--checkpoint-workload", default="gpt2")
     ap.add_argument("--zero3", action="store_true",
                     help="ZeRO-3 forward gather / release over the 7B tensor list")
     return ap.parse_args()
@@ -621,6 +625,76 @@ def run_zero3_forward(args, local_rank: int) -> dict:
             "schedule": sched.stats}
 
 
+def run_checkpoint(args, local_rank: int) -> dict:
+    """Wall-clock of `checkpoint.save` (device -> host, one file per rank, SHA-256) and
+    `checkpoint.load` (read, verify, host -> device, rebuild the half parameters) of the
+    fp32 master / exp_avg / exp_avg_sq after one step, and of a load resharded to W/2.
+    Host I/O to a temporary directory: a measurement of the host side, not of a kernel."""
+    import shutil
+    import tempfile
+
+    import torch
+
+    import synthgen
+    from synthgen import device as sdev
+    import zero_sharded_mixed_replica_b200 as zb
+    from zero_sharded_mixed_replica_b200 import checkpoint
+
+    wl = synthgen.workload(args.checkpoint_workload)
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    scaler = zb.scaler_cfg(wl.dynamic, wl.init_scale_power, wl.loss_scale_window,
+                           wl.hysteresis, wl.min_loss_scale)
+    adamw = zb.adamw_cfg(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.max_grad_norm)
+    opt = zb.ZeroOptimizer([t.shape for t in wl.tensors], wl.world, wl.bucket, wl.gdtype,
+                           wl.align, scaler, adamw, device=str(dev))
+    s = torch.cuda.current_stream(dev).cuda_stream
+    sdev.init_master(wl, opt.master, s)
+    opt.cast_params()
+    half = {"bf16": torch.bfloat16, "fp16": torch.float16}[wl.gdtype]
+    L = min(wl.bucket, opt.plan.n_pad) if wl.streaming else opt.plan.n_pad
+    grads = [torch.zeros(L, dtype=half, device=dev) for _ in range(wl.world)]
+    sdev.fill_grads(wl, grads, 0, min(L, wl.n), 1, float(2.0 ** wl.init_scale_power)
+                    if wl.dynamic else 1.0, s)
+    for b in range(opt.plan.n_buckets):
+        opt.reduce_scatter_bucket(b, grads, b * wl.bucket if wl.streaming else 0)
+    opt.step()
+    opt.result()
+    del grads
+    state_bytes = 12 * opt.plan.n_pad
+    d = tempfile.mkdtemp(prefix="zero_ckpt_")
+    try:
+        t0 = time.perf_counter()
+        checkpoint.save(opt, d)
+        t1 = time.perf_counter()
+        back = checkpoint.load(d, device=str(dev))
+        torch.cuda.synchronize(dev)
+        t2 = time.perf_counter()
+        same = all(torch.equal(a, b) for a, b in ((opt.master, back.master),
+                                                   (opt.exp_avg, back.exp_avg),
+                                                   (opt.exp_avg_sq, back.exp_avg_sq),
+                                                   (opt.params, back.params)))
+        del back
+        torch.cuda.empty_cache()
+        w2 = max(1, wl.world // 2)
+        t3 = time.perf_counter()
+        resh = checkpoint.load(d, world_size=w2, device=str(dev))
+        torch.cuda.synchronize(dev)
+        t4 = time.perf_counter()
+        n = opt.plan.n
+        same_resh = torch.equal(resh.master[:n], opt.master[:n])
+        del resh
+    finally:
+        shutil.rmtree(d, ignore_errors=True)
+    return {"mode": "checkpoint", "workload": f"{wl.name}_w{wl.world}", "params": opt.plan.n,
+            "state_bytes": state_bytes, "shards": wl.world,
+            "save_s": t1 - t0, "save_gbs": state_bytes / (t1 - t0) / 1e9,
+            "load_s": t2 - t1, "load_gbs": state_bytes / (t2 - t1) / 1e9,
+            "resharded_load_world": w2, "resharded_load_s": t4 - t3,
+            "round_trip_identical": bool(same), "resharded_identical": bool(same_resh),
+            "timing": "host wall clock (perf_counter), device synchronised"}
+
+
 # ---------------------------------------------------------------------------- oracle arm
 
 def oracle_sample_run(wl, seconds: float, max_steps: int = 0, warmup: int = 0):
@@ -709,6 +783,10 @@ def main():
 
     if args.zero3:
         print(json.dumps(run_zero3_forward(args, local_rank)), flush=True)
+        return
+
+    if args.checkpoint:
+        print(json.dumps(run_checkpoint(args, local_rank)), flush=True)
         return
 
     if args.sweep:

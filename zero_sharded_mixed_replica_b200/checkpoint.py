@@ -34,22 +34,40 @@ def _shard_name(r: int) -> str:
     return f"rank{r:05d}.bin"
 
 
+_CHUNK = 1 << 24  # bytes per hash update / write: large enough to release the GIL well
+
+
 def _sha256(path: str) -> str:
     h = hashlib.sha256()
     with open(path, "rb") as f:
-        for chunk in iter(lambda: f.read(1 << 24), b""):
+        for chunk in iter(lambda: f.read(_CHUNK), b""):
             h.update(chunk)
     return h.hexdigest()
 
 
+def _parallel(fn, items):
+    """fn over items on threads (file I/O and hashing release the GIL); in order."""
+    items = list(items)
+    if len(items) <= 1:
+        return [fn(x) for x in items]
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=min(len(items), os.cpu_count() or 1, 16)) as ex:
+        return list(ex.map(fn, items))
+
+
 def write_shard(path: str, rank: int, master: np.ndarray, exp_avg: np.ndarray,
                 exp_avg_sq: np.ndarray) -> str:
-    """One rank's partition (p elements of each array); returns the file's SHA-256."""
+    """One rank's partition (p elements of each array); returns the file's SHA-256,
+    computed over the bytes as they are written (one pass, no copy)."""
     fn = os.path.join(path, _shard_name(rank))
+    h = hashlib.sha256()
     with open(fn, "wb") as f:
         for a in (master, exp_avg, exp_avg_sq):
-            f.write(np.ascontiguousarray(a, dtype="<f4").tobytes())
-    return _sha256(fn)
+            b = memoryview(np.ascontiguousarray(a, dtype="<f4")).cast("B")
+            for i in range(0, len(b), _CHUNK):
+                h.update(b[i:i + _CHUNK])
+                f.write(b[i:i + _CHUNK])
+    return h.hexdigest()
 
 
 def write_meta(path: str, meta: dict) -> None:
@@ -77,8 +95,9 @@ def save_flat(path: str, meta_fields: dict, master: np.ndarray, exp_avg: np.ndar
     """Write all W shards and the metadata from flat n_pad arrays."""
     os.makedirs(path, exist_ok=True)
     W, p = meta_fields["world_size"], meta_fields["p"]
-    hashes = [write_shard(path, r, master[r * p:(r + 1) * p], exp_avg[r * p:(r + 1) * p],
-                          exp_avg_sq[r * p:(r + 1) * p]) for r in range(W)]
+    hashes = _parallel(lambda r: write_shard(path, r, master[r * p:(r + 1) * p],
+                                             exp_avg[r * p:(r + 1) * p],
+                                             exp_avg_sq[r * p:(r + 1) * p]), range(W))
     write_meta(path, make_meta(shard_sha256=hashes, **meta_fields))
 
 
@@ -95,15 +114,26 @@ def load_flat(path: str, verify: bool = True) -> Tuple[dict, np.ndarray, np.ndar
     meta = read_meta(path)
     W, p, n = meta["world_size"], meta["p"], meta["n"]
     out = [np.empty(W * p, np.float32) for _ in range(3)]
-    for r in range(W):
+
+    def read(r):
+        # each array's slice is read straight into place and hashed from there
         fn = os.path.join(path, meta["shards"][r])
-        if verify and _sha256(fn) != meta["sha256"][meta["shards"][r]]:
+        if os.path.getsize(fn) != 12 * p:
+            raise ValueError(f"{fn}: {os.path.getsize(fn)} bytes, expected {12 * p}")
+        h = hashlib.sha256()
+        with open(fn, "rb") as f:
+            for k in range(3):
+                b = memoryview(out[k][r * p:(r + 1) * p]).cast("B")
+                for i in range(0, len(b), _CHUNK):
+                    got = f.readinto(b[i:i + _CHUNK])
+                    if got != len(b[i:i + _CHUNK]):
+                        raise ValueError(f"{fn}: short read")
+                    if verify:
+                        h.update(b[i:i + _CHUNK])
+        if verify and h.hexdigest() != meta["sha256"][meta["shards"][r]]:
             raise ValueError(f"{fn}: checksum mismatch")
-        raw = np.fromfile(fn, dtype="<f4")
-        if raw.size != 3 * p:
-            raise ValueError(f"{fn}: {raw.size} floats, expected {3 * p}")
-        for k in range(3):
-            out[k][r * p:(r + 1) * p] = raw[k * p:(k + 1) * p]
+
+    _parallel(read, range(W))
     return meta, out[0][:n], out[1][:n], out[2][:n]
 
 
