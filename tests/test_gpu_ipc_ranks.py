@@ -6,7 +6,8 @@ update stores each rank's half values into every peer's gathered buffer (the fus
 all-gather) -- or, unfused, the slices travel through the process group. The ranks
 exchange only on the host (a device synchronize, then gloo on CPU tensors), so no
 kernel ever waits on another process's kernel. Every rank's partition state and
-gathered buffer must equal the oracle's whole-model step."""
+gathered buffer must equal the oracle's whole-model step, and a ZeRO-3 gather that reads
+the peers' partitions through the mappings must rebuild the gathered buffer."""
 import datetime
 import json
 import os
@@ -81,7 +82,15 @@ def _rank_main(rank, world, port, name, fused, out_dir):
         results.append(res)
         scale = float(res["next_scale"]) if wl.dynamic else 1.0
     torch.cuda.synchronize()
-    np.savez(os.path.join(out_dir, f"rank{rank}.npz"),
+    # ZeRO-3 gather of every tensor with the peers' partitions read through the mappings
+    # (rank q's partition is its slice of its own gathered buffer); must equal this
+    # rank's gathered buffer
+    parts = [be.peer_params[q] + 2 * q * be.p for q in range(world)]
+    gathered = torch.empty(wl.n, dtype=be.params.dtype, device="cuda")
+    zb.zero3_gather(be.plan, list(range(len(wl.tensors))), parts, gathered, s)
+    torch.cuda.synchronize()
+    zero3_ok = bool(torch.equal(gathered.view(torch.int16), be.params[:wl.n].view(torch.int16)))
+    np.savez(os.path.join(out_dir, f"rank{rank}.npz"), zero3_ok=np.array(zero3_ok),
              master=be.master.cpu().numpy(), m=be.exp_avg.cpu().numpy(),
              v=be.exp_avg_sq.cpu().numpy(), R=be.reduced.cpu().numpy(),
              params=be.params.view(torch.int16).cpu().numpy().view(np.uint16),
@@ -122,6 +131,7 @@ def test_ipc_ranks_equal_oracle(world, name, fused):
         for k in ("master", "m", "v"):
             check_state(k, got[k], ref[k][sl], 1)
         assert half_ulp_distance(got["params"], ref["params"]).max() <= 1, r
+        assert bool(got["zero3_ok"]), r
     if name == "fp16_scaler":
         assert [s["skipped"] for s in ref["scalars"]] == [0, 1, 0, 0]
     # the buffers did not start their allocations (the offsets were exercised)
