@@ -64,6 +64,10 @@ def parse_args():
     ap.add_argument("--micro", type=int, default=1,
                     help="gradient accumulation: micro-batches per step (each reduces every "
                          "bucket; the later ones add into the reduced gradient)")
+    ap.add_argument("--overlap", action="store_true",
+                    help="overlap_comm: each bucket's gradients are produced (generated) on a "
+                         "second stream while the previous bucket is reduced; timed against "
+                         "producing and reducing on one stream")
     ap.add_argument("--checkpoint", action="store_true",
                     help="sharded checkpoint save / load (and a resharded load) of the "
                          "optimizer state after one step; workload --checkpoint-workload")
@@ -625,6 +629,70 @@ def run_zero3_forward(args, local_rank: int) -> dict:
             "schedule": sched.stats}
 
 
+def run_overlap(args, local_rank: int) -> dict:
+    """ZeroOptimizer.overlapped_step on the streaming workload: bucket b's W replica
+    gradients are generated into one of two bucket-sized slots (the stand-in for the
+    backward pass producing them), then reduced. Three timings per step, CUDA events on
+    the optimizer's stream: generation and reduction on one stream (serial), on two
+    streams ordered by events (overlapped), and generation alone."""
+    import torch
+
+    from synthgen import device as sdev
+    import zero_sharded_mixed_replica_b200 as zb
+
+    wl = get_workload(args)
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cons = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(cons)
+    scaler = zb.scaler_cfg(wl.dynamic, wl.init_scale_power, wl.loss_scale_window,
+                           wl.hysteresis, wl.min_loss_scale)
+    adamw = zb.adamw_cfg(wl.lr, wl.beta1, wl.beta2, wl.eps, wl.weight_decay, wl.max_grad_norm)
+    opt = zb.ZeroOptimizer([t.shape for t in wl.tensors], wl.world, wl.bucket, wl.gdtype,
+                           wl.align, scaler, adamw, device=str(dev), stream=cons)
+    sdev.init_master(wl, opt.master, cons.cuda_stream)
+    opt.cast_params()
+    half = {"bf16": torch.bfloat16, "fp16": torch.float16}[wl.gdtype]
+    L = min(wl.bucket, opt.plan.n_pad)
+    slots = [[torch.empty(L, dtype=half, device=dev) for _ in range(wl.world)] for _ in range(2)]
+    scale = float(2.0 ** wl.init_scale_power) if wl.dynamic else 1.0
+    state = {"t": 1}
+
+    def produce(b, bufs, sh):
+        sdev.fill_grads(wl, bufs, 0, opt.plan.bucket(b)[1], state["t"], scale, sh)
+
+    def timed(prod, steps, fill_only=False):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(cons)
+        prod.wait_stream(cons)
+        for _ in range(steps):
+            if fill_only:
+                for b in range(opt.plan.n_buckets):
+                    produce(b, slots[b % 2], cons.cuda_stream)
+            else:
+                opt.overlapped_step(produce, slots, prod)
+            state["t"] += 1
+        e1.record(cons)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / steps
+
+    side = torch.cuda.Stream(dev)
+    steps = max(2, args.steps // 4)
+    timed(side, 1)  # warm-up
+    out = {"mode": "overlap_comm", "workload": f"{wl.name}_w{wl.world}", "params": opt.plan.n,
+           "buckets": opt.plan.n_buckets, "steps": steps,
+           "ms_per_step_serial": timed(cons, steps),
+           "ms_per_step_overlapped": timed(side, steps),
+           "ms_generation_only": timed(cons, steps, fill_only=True),
+           "producer": "seeded gradient generation (Philox + Irwin-Hall), ALU-bound"}
+    out["ms_hidden"] = out["ms_per_step_serial"] - out["ms_per_step_overlapped"]
+    opt.result()
+    del opt, slots
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_checkpoint(args, local_rank: int) -> dict:
     """Wall-clock of `checkpoint.save` (device -> host, one file per rank, SHA-256) and
     `checkpoint.load` (read, verify, host -> device, rebuild the half parameters) of the
@@ -787,6 +855,10 @@ def main():
 
     if args.checkpoint:
         print(json.dumps(run_checkpoint(args, local_rank)), flush=True)
+        return
+
+    if args.overlap:
+        print(json.dumps(run_overlap(args, local_rank)), flush=True)
         return
 
     if args.sweep:

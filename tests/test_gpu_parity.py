@@ -513,3 +513,30 @@ def test_binding_refuses_short_device_buffers():
         assert e.value.code == zb.ZERO_EINVAL and "needs" in e.value.message
     zb.zero_state_init(p, ws, zb.scaler_cfg(False))
     zb.zero_reduce_scatter_bucket(p, 0, "bf16", g, 0, R, ws)  # the full-size call goes through
+
+
+def test_overlapped_production_equals_serial_streaming():
+    """overlapped_step: each bucket's gradients are produced on a second stream into one
+    of two slots while the previous bucket is reduced; the result must be bit-identical
+    to producing the whole step first (the serial streaming run)."""
+    wl = synthgen.sweep(20, 4, "bf16", steps=3)
+    wl.bucket = 1 << 17  # 8 buckets
+    ref_opt, ref_res = run_streaming(wl)
+    opt = make_opt(wl)
+    s = stream()
+    sdev.init_master(wl, opt.master, s)
+    opt.cast_params()
+    slots = [[torch.empty(wl.bucket, dtype=torch.bfloat16, device="cuda") for _ in range(wl.world)]
+             for _ in range(2)]
+    prod = torch.cuda.Stream()
+    for t in range(1, wl.steps + 1):
+        def produce(b, bufs, sh, t=t):
+            sdev.fill_grads(wl, bufs, 0, opt.plan.bucket(b)[1], t, 1.0, sh)
+        opt.overlapped_step(produce, slots, prod)
+        res = opt.result()
+        assert res["global_norm"] == ref_res[t - 1]["global_norm"]
+    for a, b in ((opt.reduced, ref_opt.reduced), (opt.master, ref_opt.master),
+                 (opt.exp_avg, ref_opt.exp_avg), (opt.exp_avg_sq, ref_opt.exp_avg_sq),
+                 (opt.params, ref_opt.params)):
+        assert torch.equal(a.view(torch.int32 if a.element_size() == 4 else torch.int16),
+                           b.view(torch.int32 if b.element_size() == 4 else torch.int16))

@@ -106,6 +106,32 @@ class ZeroOptimizer:
             self.reduce_scatter_bucket(b, replica_grads, base_offset)
         self.step()
 
+    def overlapped_step(self, produce, slots: Sequence[Sequence], producer_stream) -> None:
+        """One step whose reduce-scatter of bucket b overlaps the production of the next
+        buckets (the pages' overlap_comm). `produce(b, bufs, stream)` enqueues on `stream`
+        (the producer's, a raw handle) the writes of bucket b's W replica gradients into
+        `bufs`, one of the `slots` (each a list of W buffers of at least one bucket,
+        indexed from the bucket start). Bucket b goes to slot b % len(slots); it is reduced
+        on this optimizer's stream as soon as it has been written, and the slot goes back
+        to the producer once the reduction has read it. With two slots the reduction of
+        bucket b runs while bucket b + 1 is produced. Events order the two streams; the
+        host never waits."""
+        cons = self.stream if self.stream is not None else torch.cuda.current_stream(self.device)
+        n = len(slots)
+        ev = getattr(self, "_slot_events", None)
+        if ev is None or len(ev) != n:
+            ev = self._slot_events = [(torch.cuda.Event(), torch.cuda.Event()) for _ in range(n)]
+        for b in range(self.plan.n_buckets):
+            ready, free = ev[b % n]
+            producer_stream.wait_event(free)  # the slot's previous bucket has been read
+            with torch.cuda.stream(producer_stream):
+                produce(b, slots[b % n], producer_stream.cuda_stream)
+            ready.record(producer_stream)
+            cons.wait_event(ready)
+            self.reduce_scatter_bucket(b, slots[b % n], base_offset=self.plan.bucket(b)[0])
+            free.record(cons)
+        self.step()
+
     def capture_step(self, replica_grads: Sequence, base_offset: int = 0) -> torch.cuda.CUDAGraph:
         """A CUDA graph of one full step over fixed replica buffers (every launch of the
         step, no host work): `graph.replay()` runs a step. The step allocates nothing and
