@@ -438,7 +438,6 @@ def run_e2e(args, wl, local_rank: int, world_size: int = 1):
     with CUDA events on the stream that carries the copies, the kernels and the result
     read (host waits between steps show up as idle time); max over ranks. With several
     ranks each keeps one pinned slot (every step reuses it) to bound host memory."""
-    import numpy as np
     import torch
 
     import synthgen
@@ -463,11 +462,16 @@ def run_e2e(args, wl, local_rank: int, world_size: int = 1):
     n_slots = 2 if world_size == 1 else 1
     host = [[torch.zeros(L, dtype=torch.int16).pin_memory() for _ in range(W)]
             for _ in range(n_slots)]
+    # generated on the device (the same bits as the host generator) and copied into the
+    # pinned buffers: seconds instead of a minute of host arithmetic per rank
+    tmp = torch.zeros(L, dtype=torch.int16, device=dev)
     for k in range(n_slots):
         for r in range(W):
-            synthgen.grads_host(0, min(L, wl.n), wl.seed, r, wl.slot(k + 1), wl.grad_sigma,
-                                wl.spike_frac, 1.0, wl.dtype_code,
-                                out=host[k][r].numpy().view(np.uint16))
+            synthgen.grads_cuda(tmp.data_ptr(), 0, min(L, wl.n), wl.seed, r, wl.slot(k + 1),
+                                wl.grad_sigma, wl.spike_frac, 1.0, wl.dtype_code, s.cuda_stream)
+            host[k][r].copy_(tmp)
+    torch.cuda.synchronize(dev)
+    del tmp
     staging = [torch.empty(min(wl.bucket, plan.n_pad), dtype=half, device=dev) for _ in range(W)]
     h2d = 0
 
