@@ -85,6 +85,24 @@ def get_workload(args):
     return wl
 
 
+def workload_config(wl, n_buckets: int, n_pad: int, world_size: int, micro: int = 1) -> dict:
+    """The `config` object of the JSON line (both arms describe the same workload)."""
+    step_bytes = (schedule_bytes_per_param(wl.world) + (micro - 1) * (2 * wl.world + 8)) * n_pad
+    return {
+        "workload": f"{wl.name}_w{wl.world}",
+        "params": wl.n,
+        "tensors": len(wl.tensors),
+        "W": wl.world,
+        "reduce_bucket_size": wl.bucket,
+        "buckets": n_buckets,
+        "grad_dtype": wl.gdtype,
+        "replica_buffers": "bucket-sized, 2 slots" if wl.streaming else "resident",
+        "micro_batches": micro,
+        "l2": f"no flush: each step moves {step_bytes / 1e9:.0f} GB, inputs >> 126 MB L2",
+        "parallelism": f"replicas x{world_size} (simulated dp{wl.world} per GPU)",
+    }
+
+
 def schedule_bytes_per_param(W: int) -> int:
     # reduce-scatter: W half reads + fp32 write; update: fp32 R, p, m, v reads, p, m, v
     # writes and the half write
@@ -379,19 +397,7 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
             "vs_baseline": None,
             "dtype": "f32",  # arithmetic of the step (half inputs, fp64 norm)
             "data": "synthetic (seeded Philox gradients and init; random-init weights of the shape list)",
-            "config": {
-                "workload": f"{wl.name}_w{W}",
-                "params": plan.n,
-                "tensors": len(wl.tensors),
-                "W": W,
-                "reduce_bucket_size": wl.bucket,
-                "buckets": nb,
-                "grad_dtype": wl.gdtype,
-                "replica_buffers": "bucket-sized, 2 slots" if wl.streaming else "resident",
-                "micro_batches": M,
-                "l2": f"no flush: each step moves {step_bytes / 1e9:.0f} GB, inputs >> 126 MB L2",
-                "parallelism": f"replicas x{world_size} (simulated dp{W} per GPU)",
-            },
+            "config": workload_config(wl, nb, n_pad, world_size, M),
             "hbm_gbs_schedule": sched_gbs,
             "hbm_gbs_model": model_gbs,
             "frac_of_8tbs_schedule": sched_gbs / 8000.0,
@@ -813,10 +819,12 @@ def oracle_sample_run(wl, seconds: float, max_steps: int = 0, warmup: int = 0):
     return n * steps / el, desc, steps, el
 
 
-def run_reference(args, rank: int):
+def run_reference(args, rank: int, world_size: int = 1):
     if rank != 0:
         return None
+    import oracle
     wl = get_workload(args)
+    pl = oracle.plan(wl.numels, wl.world, wl.bucket, wl.align)
     val, desc, steps, el = oracle_sample_run(wl, 0, max_steps=args.steps, warmup=args.warmup)
     return {
         "impl": "reference",
@@ -832,8 +840,7 @@ def run_reference(args, rank: int):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic (seeded Philox gradients and init)",
-        "config": {"workload": f"{wl.name}_w{wl.world}", "params": wl.n, "W": wl.world,
-                   "reduce_bucket_size": wl.bucket},
+        "config": workload_config(wl, pl.n_buckets, pl.n_pad, world_size, max(1, args.micro)),
         "cpu_baseline": {"value": val, "unit": "params/s", "cores": 1, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": val, "unit": "params/s", "h2d_bytes_per_step": 0,
@@ -848,7 +855,7 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
     if args.impl == "reference":
-        out = run_reference(args, rank)
+        out = run_reference(args, rank, world_size)
         if out is not None:
             print(json.dumps(out), flush=True)
         return
