@@ -151,3 +151,17 @@ def test_distributed_step_equals_single_process(world, name):
                 assert np.array_equal(got[k], ref[k][sl]), (r, k)
         if name == "fp16_scaler":
             assert list(ranks[0]["skipped"]) == [0, 1, 1, 0, 0]
+
+
+def test_allgather_chunks_cover_the_partition():
+    from zero_sharded_mixed_replica_b200.distributed import allgather_chunks
+    assert allgather_chunks(0, 5) == []
+    assert allgather_chunks(10, None) == [(0, 10)]
+    assert allgather_chunks(10, 10) == [(0, 10)] == allgather_chunks(10, 99)
+    assert allgather_chunks(10, 3) == [(0, 3), (3, 6), (6, 9), (9, 10)]
+    for p in range(1, 60):
+        for b in range(1, 70):
+            ch = allgather_chunks(p, b)
+            assert ch[0][0] == 0 and ch[-1][1] == p
+            assert all(a1 == b0 for (_, a1), (b0, _) in zip(ch, ch[1:]))
+            assert all(0 < e - s <= b for s, e in ch)

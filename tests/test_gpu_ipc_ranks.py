@@ -40,7 +40,7 @@ def _workload(name, world):
         inf_sites={2: 1})
 
 
-def _rank_main(rank, world, port, name, fused, out_dir):
+def _rank_main(rank, world, port, name, fused, out_dir, ag_bucket=None):
     import torch.distributed as dist
 
     from synthgen import device as sdev
@@ -60,7 +60,7 @@ def _rank_main(rank, world, port, name, fused, out_dir):
     pad = torch.zeros(4096 * (rank + 1), dtype=torch.uint8, device="cuda")
     be = CudaRankBackend([t.shape for t in wl.tensors], wl.bucket, wl.gdtype, rank, world,
                          align=wl.align, scaler=scaler, adamw=adamw, fused_all_gather=fused,
-                         host_exchange=True)
+                         host_exchange=True, allgather_bucket_size=ag_bucket)
     s = torch.cuda.current_stream().cuda_stream
     full = torch.zeros(be.n_pad, dtype=torch.float32, device="cuda")
     sdev.init_master(wl, full, s)
@@ -110,14 +110,16 @@ def _free_port():
     return port
 
 
-@pytest.mark.parametrize("world,name,fused", [(2, "bf16_ragged", True), (3, "bf16_ragged", True),
-                                              (2, "fp16_scaler", True),
-                                              (2, "bf16_ragged", False)],
-                         ids=["w2_bf16_fused", "w3_bf16_fused", "w2_fp16_fused", "w2_bf16_gather_via_group"])
-def test_ipc_ranks_equal_oracle(world, name, fused):
+@pytest.mark.parametrize("world,name,fused,ag_bucket",
+                         [(2, "bf16_ragged", True, None), (3, "bf16_ragged", True, None),
+                          (2, "fp16_scaler", True, None), (2, "bf16_ragged", False, None),
+                          (3, "bf16_ragged", False, 10000)],
+                         ids=["w2_bf16_fused", "w3_bf16_fused", "w2_fp16_fused",
+                              "w2_bf16_gather_via_group", "w3_bf16_gather_in_buckets"])
+def test_ipc_ranks_equal_oracle(world, name, fused, ag_bucket):
     with tempfile.TemporaryDirectory() as d:
-        mp.start_processes(_rank_main, args=(world, _free_port(), name, fused, d), nprocs=world,
-                           join=True, start_method="spawn")
+        mp.start_processes(_rank_main, args=(world, _free_port(), name, fused, d, ag_bucket),
+                           nprocs=world, join=True, start_method="spawn")
         ranks = [dict(np.load(os.path.join(d, f"rank{r}.npz"))) for r in range(world)]
     wl = _workload(name, world)
     ref = oracle.run_resident(wl)

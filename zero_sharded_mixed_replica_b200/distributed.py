@@ -21,7 +21,7 @@ insight (each GPU keeps only its own gradient slice).
 """
 from __future__ import annotations
 
-from typing import Dict, List, Optional, Sequence
+from typing import Dict, List, Optional, Sequence, Tuple
 
 import torch
 import torch.distributed as dist
@@ -32,6 +32,16 @@ from . import (AdamWCfg, Plan, ScalerCfg, adamw_cfg, scaler_cfg, zero_get_result
                zero_step_local_sumsq, zero_step_update_partition)
 
 _TORCH_HALF = {"bf16": torch.bfloat16, "fp16": torch.float16}
+
+
+def allgather_chunks(p: int, allgather_bucket_size: Optional[int]) -> List[Tuple[int, int]]:
+    """[start, end) ranges of a partition of p elements gathered one bucket at a time
+    ([Z2] ds_config allgather_bucket_size, counted in elements like reduce_bucket_size);
+    None or a size >= p gathers the partition at once."""
+    if p <= 0:
+        return []
+    b = p if not allgather_bucket_size or allgather_bucket_size >= p else int(allgather_bucket_size)
+    return [(c, min(c + b, p)) for c in range(0, p, b)]
 
 
 def partition_buckets(plan_n_pad: int, world: int, bucket: int, rank: int) -> range:
@@ -79,7 +89,7 @@ class CudaRankBackend:
                  rank: int, world: int, group=None, align: int = 128,
                  scaler: Optional[ScalerCfg] = None, adamw: Optional[AdamWCfg] = None,
                  fused_all_gather: bool = True, device: Optional[torch.device] = None,
-                 host_exchange: bool = False):
+                 host_exchange: bool = False, allgather_bucket_size: Optional[int] = None):
         self.rank, self.world, self.dtype = rank, world, dtype
         self.device = device or torch.device("cuda", torch.cuda.current_device())
         self.plan = Plan(shapes, world, reduce_bucket_size, align)
@@ -98,6 +108,7 @@ class CudaRankBackend:
         self.adamw = adamw if adamw is not None else adamw_cfg()
         self.fused_all_gather = fused_all_gather
         self.host_exchange = host_exchange
+        self.gather_chunks = allgather_chunks(self.p, allgather_bucket_size)
         zero_state_init(self.plan, self.workspace, self.scaler, self._s())
         # peers' buffers, mapped once (IPC handles travel through the process group). A
         # handle names a whole allocation, which may hold both buffers: each distinct
@@ -173,12 +184,18 @@ class CudaRankBackend:
     def after_update(self, group) -> None:
         if self.host_exchange:
             if not self.fused_all_gather:
-                # the half slices travel as bytes (gloo has no 16-bit float types)
+                # one bucket of every rank's slice at a time; the halves travel as bytes
+                # (gloo has no 16-bit float types)
                 own = self.own_slice().cpu().view(torch.uint8)
-                parts = [torch.empty_like(own) for _ in range(self.world)]
-                dist.all_gather(parts, own, group=group)
-                self.params.copy_(torch.cat(parts).view(self.params.dtype).to(self.device))
-            # the peers' stores into this buffer (or the copy above) have landed, and
+                for c0, c1 in self.gather_chunks:
+                    parts = [torch.empty(2 * (c1 - c0), dtype=torch.uint8)
+                             for _ in range(self.world)]
+                    dist.all_gather(parts, own[2 * c0:2 * c1].contiguous(), group=group)
+                    for q, part in enumerate(parts):
+                        lo = q * self.p
+                        self.params[lo + c0:lo + c1].copy_(
+                            part.view(self.params.dtype).to(self.device))
+            # the peers' stores into this buffer (or the copies above) have landed, and
             # every rank is done reading the peers' gradients
             self._host_barrier(group)
             return
@@ -187,8 +204,13 @@ class CudaRankBackend:
             # rank uses its buffer
             flag = torch.zeros(1, device=self.device)
             dist.all_reduce(flag, group=group)
-        else:
+        elif len(self.gather_chunks) == 1:
             dist.all_gather_into_tensor(self.params, self.own_slice().clone(), group=group)
+        else:
+            own = self.own_slice().clone()
+            for c0, c1 in self.gather_chunks:
+                dist.all_gather([self.params[q * self.p + c0:q * self.p + c1]
+                                 for q in range(self.world)], own[c0:c1], group=group)
 
     def result(self) -> dict:
         return zero_get_result(self.workspace, self._s())
