@@ -540,3 +540,16 @@ def test_overlapped_production_equals_serial_streaming():
                  (opt.params, ref_opt.params)):
         assert torch.equal(a.view(torch.int32 if a.element_size() == 4 else torch.int16),
                            b.view(torch.int32 if b.element_size() == 4 else torch.int16))
+
+
+def test_all_gather_tma_ring_wraps():
+    """Enough 32 KB tiles that every CTA of the copy kernel wraps its 4-stage ring, a
+    ragged tail after the last full tile, and two launches of destinations."""
+    n = 148 * 16384 * 6 + 12345
+    opt = zb.ZeroOptimizer([(n,)], 2, 1 << 30, align=1)
+    src = torch.randint(-32768, 32767, (opt.plan.n_pad,), dtype=torch.int16, device="cuda")
+    opt.params.view(torch.int16).copy_(src)
+    dst = [torch.zeros_like(opt.params) for _ in range(17)]
+    opt.all_gather(dst)
+    for d in dst:
+        assert torch.equal(d.view(torch.int16), src)

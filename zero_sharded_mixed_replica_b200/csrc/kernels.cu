@@ -140,6 +140,20 @@ __device__ __forceinline__ void bulk_load(void* dst_smem, const void* src, uint3
       : "memory");
 }
 
+// 1-D bulk copy shared -> global (TMA store), tracked by bulk async-groups of this thread
+__device__ __forceinline__ void bulk_store(void* dst, const void* src_smem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_addr(src_smem)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// at most one committed group still reading its shared-memory source
+__device__ __forceinline__ void bulk_wait_read_but1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+// every committed group complete (its writes performed)
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ------------------------------------------------------------------ half helpers
 
 // dtype 0 = bf16, 1 = fp16
@@ -714,16 +728,80 @@ struct ReplicateArgs {
   int64_t n;
 };
 
-__global__ void __launch_bounds__(kUpThreads) replicate_kernel(const __grid_constant__ ReplicateArgs a) {
-  const int64_t nthr = (int64_t)gridDim.x * kUpThreads;
-  const int64_t tid = (int64_t)blockIdx.x * kUpThreads + threadIdx.x;
-  const int64_t nvec = a.n / 8;
-  for (int64_t vi = tid; vi < nvec; vi += nthr) {
-    const uint4 x = ld_nc_u4(a.src + vi * 8);
-    for (int d = 0; d < a.n_dst; ++d) st_u4(a.dst[d] + vi * 8, x.x, x.y, x.z, x.w);
+// K4: copies of the gathered buffer into per-rank buffers, moved by the TMA engine alone.
+// Thread 0 of each CTA bulk-loads 32 KB tiles (tile blockIdx + j * gridDim) into a
+// 4-stage shared-memory ring and bulk-stores each landed tile to every destination (one
+// bulk group per tile); a stage is reloaded once the stores of its previous tile have read
+// it. The elements after the last full tile are copied by the last CTA's warp. A load
+// wait that gives up (about one second) ends the ring; the CTA then waits (bounded) for
+// its copies in flight and copies its remaining tiles with plain loads, so the result
+// stays complete. Sources and destinations are 16-byte aligned (checked by the caller).
+constexpr int kRepStages = 4;
+constexpr int kRepTileBytes = 32768;
+constexpr int kRepThreads = 32;
+constexpr size_t kRepSmemBytes = (size_t)kRepStages * kRepTileBytes + kRepStages * sizeof(uint64_t);
+
+__global__ void __launch_bounds__(kRepThreads) replicate_kernel(const __grid_constant__ ReplicateArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t* full = (uint64_t*)(smem + (size_t)kRepStages * kRepTileBytes);
+  __shared__ int64_t first_plain;  // first of this CTA's tiles left to the plain copy
+  constexpr int64_t kTileElems = kRepTileBytes / 2;
+  const int64_t n_tiles = a.n / kTileElems;
+  const int64_t G = gridDim.x;
+  const int64_t my = (int64_t)blockIdx.x < n_tiles ? (n_tiles - blockIdx.x + G - 1) / G : 0;
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kRepStages; ++st) mbar_init(&full[st], 1);
+    mbar_init_fence();
+    int64_t issued = my < kRepStages ? my : kRepStages;
+    for (int64_t j = 0; j < issued; ++j) {
+      mbar_arrive_expect_tx(&full[j], kRepTileBytes);
+      bulk_load(smem + j * kRepTileBytes, a.src + (blockIdx.x + j * G) * kTileElems,
+                kRepTileBytes, &full[j]);
+    }
+    int64_t j = 0;
+    for (; j < my; ++j) {
+      const int st = (int)(j % kRepStages);
+      if (!mbar_wait(&full[st], (uint32_t)((j / kRepStages) & 1))) break;
+      const int64_t off = (blockIdx.x + j * G) * kTileElems;
+      for (int d = 0; d < a.n_dst; ++d)
+        bulk_store(a.dst[d] + off, smem + st * kRepTileBytes, kRepTileBytes);
+      bulk_commit();
+      if (j >= 1) {
+        bulk_wait_read_but1();  // the stores of tile j - 1 have read their stage
+        const int64_t jn = j - 1 + kRepStages;
+        if (jn < my) {
+          const int sp = (int)(jn % kRepStages);
+          mbar_arrive_expect_tx(&full[sp], kRepTileBytes);
+          bulk_load(smem + sp * kRepTileBytes, a.src + (blockIdx.x + jn * G) * kTileElems,
+                    kRepTileBytes, &full[sp]);
+          issued = jn + 1;
+        }
+      }
+    }
+    // loads still in flight (only after a wait gave up) land before the CTA goes on
+    for (int64_t q = j; q < issued; ++q)
+      mbar_wait(&full[q % kRepStages], (uint32_t)((q / kRepStages) & 1));
+    bulk_wait_all();
+    first_plain = j;
   }
-  for (int64_t i = nvec * 8 + tid; i < a.n; i += nthr)
-    for (int d = 0; d < a.n_dst; ++d) a.dst[d][i] = a.src[i];
+  __syncwarp();
+  for (int64_t j = first_plain; j < my; ++j) {  // empty unless a wait gave up
+    const int64_t off = (blockIdx.x + j * G) * kTileElems;
+    for (int64_t v = threadIdx.x; v < kTileElems / 8; v += kRepThreads) {
+      const uint4 x = ld_nc_u4(a.src + off + v * 8);
+      for (int d = 0; d < a.n_dst; ++d) st_u4(a.dst[d] + off + v * 8, x.x, x.y, x.z, x.w);
+    }
+  }
+  if (blockIdx.x == G - 1) {  // the elements after the last full tile
+    const int64_t t0 = n_tiles * kTileElems;
+    const int64_t nvec = (a.n - t0) / 8;
+    for (int64_t v = threadIdx.x; v < nvec; v += kRepThreads) {
+      const uint4 x = ld_nc_u4(a.src + t0 + v * 8);
+      for (int d = 0; d < a.n_dst; ++d) st_u4(a.dst[d] + t0 + v * 8, x.x, x.y, x.z, x.w);
+    }
+    for (int64_t i = t0 + nvec * 8 + threadIdx.x; i < a.n; i += kRepThreads)
+      for (int d = 0; d < a.n_dst; ++d) a.dst[d][i] = a.src[i];
+  }
 }
 
 __global__ void state_init_kernel(WsHeader* h, zero_scaler_cfg cfg) {
@@ -996,10 +1074,15 @@ cudaError_t launch_cast(int dtype, const float* master, void* params, int64_t n,
 cudaError_t launch_replicate(const void* src, void* const* dst, int n_dst, int64_t n_halves,
                              cudaStream_t s) {
   if (n_halves == 0 || n_dst == 0) return cudaSuccess;
-  int grid = 1;
-  cudaError_t e = persistent_grid((const void*)replicate_kernel, kUpThreads,
-                                  (n_halves + 7) / 8, &grid);
+  cudaError_t e = cudaFuncSetAttribute((const void*)replicate_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kRepSmemBytes);
   if (e != cudaSuccess) return e;
+  // one CTA per SM (the ring takes 128 KB of shared memory), never more than the tiles
+  const int64_t n_tiles = n_halves / (kRepTileBytes / 2);
+  int64_t grid = sm_count();
+  if (grid > n_tiles) grid = n_tiles;
+  if (grid < 1) grid = 1;
   for (int d0 = 0; d0 < n_dst; d0 += kReplicateMax) {
     ReplicateArgs a;
     a.src = (const uint16_t*)src;
@@ -1008,7 +1091,8 @@ cudaError_t launch_replicate(const void* src, void* const* dst, int n_dst, int64
       a.dst[d] = d < a.n_dst ? (uint16_t*)dst[d0 + d] : nullptr;
     a.n = n_halves;
     void* args[] = {&a};
-    e = cudaLaunchKernel((const void*)replicate_kernel, dim3(grid), dim3(kUpThreads), args, 0, s);
+    e = cudaLaunchKernel((const void*)replicate_kernel, dim3((unsigned)grid), dim3(kRepThreads),
+                         args, kRepSmemBytes, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
