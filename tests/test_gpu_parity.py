@@ -382,10 +382,11 @@ def _check_streaming(wl, idx=None, steps=None):
     return results
 
 
-@pytest.mark.parametrize("world,dtype", [(1, "bf16"), (16, "bf16"), (1, "fp16"), (16, "fp16")])
+@pytest.mark.parametrize("world", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
 def test_sweep_2_24_every_element(world, dtype):
-    """Sweep point 2^24 x W x dtype, 10 steps (fp16: dynamic scaler with one +inf at
-    step 5), every element compared."""
+    """Every 2^24 sweep point (W in {1, 2, 4, 8, 16} x {bf16, fp16}), 10 steps (fp16:
+    dynamic scaler with one +inf at step 5), every element compared."""
     wl = synthgen.sweep(24, world, dtype)
     results = _check_streaming(wl)
     if dtype == "fp16":
