@@ -85,6 +85,25 @@ def get_workload(args):
     return wl
 
 
+def max_over_ranks(x: float, world_size: int, device) -> float:
+    """The largest of every rank's x (the job's time is its slowest rank's). A collective
+    of the default process group on `device` (a CUDA device under NCCL, "cpu" under gloo);
+    every rank calls it in the same order."""
+    if world_size <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step: int, steps: int, world_size: int, seconds: float) -> float:
+    """Units processed by all ranks per second of the slowest rank (weak scaling: every
+    rank runs the same workload)."""
+    return units_per_rank_step * steps * world_size / seconds
+
+
 def workload_config(wl, n_buckets: int, n_pad: int, world_size: int, micro: int = 1) -> dict:
     """The `config` object of the JSON line (both arms describe the same workload)."""
     step_bytes = (schedule_bytes_per_param(wl.world) + (micro - 1) * (2 * wl.world + 8)) * n_pad
@@ -350,17 +369,13 @@ def run_ours(args, rank: int, world_size: int, local_rank: int):
     else:  # no events inside a graph: only whole steps are timed
         k1_ms = k2_ms = k3_ms = [float("nan")]
 
-    ms_max = ms_total
-    if world_size > 1:
-        tt = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_max = float(tt.item())
+    ms_max = max_over_ranks(ms_total, world_size, dev)
 
     out = None
     if rank == 0:
         ms_step = ms_max / args.steps
         params_step = plan.n  # parameters updated per step (padding excluded)
-        value = params_step * args.steps * world_size / (ms_max / 1e3)
+        value = whole_job_rate(params_step, args.steps, world_size, ms_max / 1e3)
         peak, peak_kind = measured_peaks()
         k3_avg = sum(k3_ms) / len(k3_ms)
         k3_bytes = 30 * n_pad  # R, p, m, v read (16 B) + p, m, v write (12 B) + half (2 B)
@@ -503,12 +518,8 @@ def run_e2e(args, wl, local_rank: int, world_size: int = 1):
         one(i + 2)
     e1.record(s)
     torch.cuda.synchronize(dev)
-    dt = e0.elapsed_time(e1) / 1e3
-    if world_size > 1:
-        tt = torch.tensor([dt], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        dt = float(tt.item())
-    out = {"value": plan.n * args.e2e_steps * world_size / dt, "unit": "params/s",
+    dt = max_over_ranks(e0.elapsed_time(e1) / 1e3, world_size, dev)
+    out = {"value": whole_job_rate(plan.n, args.e2e_steps, world_size, dt), "unit": "params/s",
            "h2d_bytes_per_step": h2d // args.e2e_steps,
            "d2h_bytes_per_step": ctypes.sizeof(zb.StepResult),
            "steps": args.e2e_steps,
