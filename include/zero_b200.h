@@ -38,7 +38,11 @@
  *    the stream. The library owns only the plan (host memory). It never allocates
  *    device memory and never synchronises, except zero_get_result.
  *  - Streams: `stream` is a cudaStream_t passed as void*; NULL is the legacy default
- *    stream. All device work of a call is enqueued on that stream, in order.
+ *    stream. All device work of a call is enqueued on that stream, in order. The step
+ *    kernels (bucket reduction, finalize, update) are launched with programmatic stream
+ *    serialization: one may be scheduled while the kernel before it in the stream is
+ *    finishing, but it reads and writes no global memory until that kernel has
+ *    completed, so stream order holds exactly as for ordinary launches.
  *  - Device pointers must be 16-byte aligned (ZERO_EALIGN otherwise).
  *  - Conditions found on the device (overflow, a skipped step) are results, not errors.
  *  - Calls on one plan must not run concurrently from several host threads.
