@@ -59,6 +59,9 @@ def parse_args():
     ap.add_argument("--sweep-log2n", default="24,26,28,30")
     ap.add_argument("--sweep-world", default="1,2,4,8,16")
     ap.add_argument("--sweep-dtype", default="bf16,fp16")
+    ap.add_argument("--resident", action="store_true",
+                    help="sweep: points with W <= 2 keep whole-model replica buffers and run "
+                         "zero_step_resident (4W + 26 bytes per parameter)")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step from a CUDA graph (launch-bound small workloads)")
     ap.add_argument("--micro", type=int, default=1,
@@ -529,10 +532,12 @@ def run_e2e(args, wl, local_rank: int, world_size: int = 1):
     return out
 
 
-def run_sweep_point(wl, steps: int, local_rank: int) -> dict:
+def run_sweep_point(wl, steps: int, local_rank: int, resident: bool = False) -> dict:
     """All steps of one sweep point. Replica slots are regenerated before every step
     (the loss scale in force for fp16, the +inf site at step 5) outside the timed part;
-    each step's kernels are timed with CUDA events on the launching stream."""
+    each step's kernels are timed with CUDA events on the launching stream. With
+    `resident` (W <= 2 only) the replicas cover the whole flat space and the step is
+    zero_step_resident."""
     import torch
 
     from synthgen import device as sdev
@@ -551,31 +556,44 @@ def run_sweep_point(wl, steps: int, local_rank: int) -> dict:
     plan = opt.plan
     sdev.init_master(wl, opt.master, sh)
     opt.cast_params()
-    L = min(wl.bucket, plan.n_pad)
-    slots = [[torch.empty(L, dtype=half, device=dev) for _ in range(wl.world)] for _ in range(2)]
+    resident = resident and wl.world <= 2
+    L = plan.n_pad if resident else min(wl.bucket, plan.n_pad)
+    slots = [[torch.empty(L, dtype=half, device=dev) for _ in range(wl.world)]
+             for _ in range(1 if resident else 2)]
     scale = float(2.0 ** wl.init_scale_power) if wl.dynamic else 1.0
+    inf_bits = torch.tensor(0x7C00 if wl.gdtype == "fp16" else 0x7F80,
+                            dtype=torch.int32).to(torch.int16)
     applied, skipped = [], []
     for t in range(1, steps + 1):
-        bufs = slots[(t - 1) % 2]
+        bufs = slots[(t - 1) % len(slots)]
         sdev.fill_grads(wl, bufs, 0, L, t, scale, sh)
-        sdev.plant_infs(wl, bufs, t, wl.bucket)
+        if resident:  # the +inf sites at their flat index
+            for idx, rep in wl.inf_sites_at(t):
+                bufs[rep].view(torch.int16)[idx] = inf_bits
+        else:
+            sdev.plant_infs(wl, bufs, t, wl.bucket)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(s)
-        for bk in range(plan.n_buckets):
-            opt.reduce_scatter_bucket(bk, bufs, base_offset=bk * wl.bucket)
-        opt.step()
+        if resident:
+            opt.step_resident(bufs)
+        else:
+            for bk in range(plan.n_buckets):
+                opt.reduce_scatter_bucket(bk, bufs, base_offset=bk * wl.bucket)
+            opt.step()
         b.record(s)
         res = opt.result()
         (skipped if res["skipped"] else applied).append(a.elapsed_time(b))
         scale = float(res["next_scale"]) if wl.dynamic else 1.0
     ms = statistics.median(applied[1:] if len(applied) > 2 else applied)
     W = wl.world
+    sched = 4 * W + 26 if resident else schedule_bytes_per_param(W)
     out = {
         "point": wl.name, "params": plan.n, "W": W, "grad_dtype": wl.gdtype,
         "buckets": plan.n_buckets, "steps": steps,
+        "schedule": "resident replicas (4W+26 B/param)" if resident else "stored R (2W+34 B/param)",
         "ms_per_applied_step_median": ms,
         "params_per_s": plan.n / (ms / 1e3),
-        "hbm_gbs_schedule": schedule_bytes_per_param(W) * plan.n_pad / (ms / 1e3) / 1e9,
+        "hbm_gbs_schedule": sched * plan.n_pad / (ms / 1e3) / 1e9,
         "hbm_gbs_model": model_bytes_per_param(W) * plan.n / (ms / 1e3) / 1e9,
         "first_step_ms": (applied + skipped)[0],
         "skipped_steps": len(skipped),
@@ -889,7 +907,8 @@ def main():
             for W in [int(x) for x in args.sweep_world.split(",")]:
                 for dt in args.sweep_dtype.split(","):
                     wl = synthgen.sweep(log2n, W, dt)
-                    print(json.dumps(run_sweep_point(wl, wl.steps, local_rank)), flush=True)
+                    print(json.dumps(run_sweep_point(wl, wl.steps, local_rank, args.resident)),
+                          flush=True)
         return
 
     import torch

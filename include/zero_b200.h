@@ -282,6 +282,25 @@ ZERO_API int zero_step_update(zero_plan* plan, float* master, float* exp_avg, fl
                      const float* reduced, void* params, int32_t param_dtype,
                      const void* workspace, void* stream);
 
+/* zero_step_resident: the whole step for W <= 2 ranks whose replica gradients are all
+ * still in device memory when the step runs ([Z1] 2.1 the reduce-scatter of gradients
+ * and the per-partition update; the schedule is this library's). The bucket kernel
+ * computes only the sum of squares of every bucket (no reduced gradient is stored),
+ * and the update forms each element's reduced gradient again from the replicas -- the
+ * same rank-ordered fp32 sum, so every result is bit-identical to
+ * zero_reduce_scatter_bucket for each bucket followed by zero_step. It moves 4W + 26
+ * bytes per parameter instead of 2W + 34: 30 against 36 at W = 1, 34 against 38 at
+ * W = 2 (equal at W = 4, more above; hence the limit).
+ *   replica_grads[r]: replica r's gradients over the whole padded flat space (n_pad
+ *       elements of grad_dtype, 16-byte aligned); master / exp_avg / exp_avg_sq: fp32,
+ *       n_pad elements; params: the gathered buffer, n_pad elements of param_dtype.
+ * Errors: EINVAL (NULL, bad dtype or hyperparameters, world_size > 2), EALIGN, ESTATE
+ * when buckets of this step were already reduce-scattered, ECUDA. */
+ZERO_API int zero_step_resident(zero_plan* plan, const zero_adamw_cfg* cfg, int32_t grad_dtype,
+                                const void* const* replica_grads, float* master,
+                                float* exp_avg, float* exp_avg_sq, void* params,
+                                int32_t param_dtype, void* workspace, void* stream);
+
 /* zero_all_gather ([Z1] 2.1 parameters gathered by allgather; [Z1] 2.2 batched
  * all-gather; [Z2] allgather_bucket_size): after zero_step the gathered buffer `params`
  * already holds every rank's partition, so n_dst = 0 is a no-op. With n_dst > 0 the

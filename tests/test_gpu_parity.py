@@ -554,3 +554,56 @@ def test_all_gather_tma_ring_wraps():
     opt.all_gather(dst)
     for d in dst:
         assert torch.equal(d.view(torch.int16), src)
+
+
+# ----------------------------------------------------------------------------- resident W <= 2
+
+RESIDENT = [
+    ([(1 << 20,)], 2, 1 << 20, 128, "bf16", False, 3),             # the tiny shape, one bucket
+    ([(300001,), (77, 5)], 1, 65536, 8, "bf16", False, 3),         # W=1, several buckets, tail
+    ([(4097,), (129, 3), (50000,)], 2, 1001, 1, "fp16", True, 4),  # fp16 scaler, +inf at step 2
+]
+
+
+@pytest.mark.parametrize("case", RESIDENT, ids=["w2_bf16", "w1_ragged", "w2_fp16_overflow"])
+def test_step_resident_equals_oracle(case):
+    """zero_step_resident (sum of squares only in the bucket kernel; the update sums the
+    resident replicas again) against the oracle's step: same bits as the stored-R path."""
+    wl = _edge_workload(*case)
+    ref = oracle.run_resident(wl)
+    opt = make_opt(wl)
+    s = stream()
+    sdev.init_master(wl, opt.master, s)
+    opt.cast_params()
+    n_pad = opt.plan.n_pad
+    grads = [torch.zeros(n_pad, dtype=HALF[wl.gdtype], device="cuda") for _ in range(wl.world)]
+    scale = float(2.0 ** wl.init_scale_power) if wl.dynamic else 1.0
+    for t in range(1, wl.steps + 1):
+        sdev.fill_grads(wl, grads, 0, wl.n, t, scale, s)
+        sdev.plant_infs(wl, grads, t)
+        opt.step_resident(grads)
+        res = opt.result()
+        check_scalars(res, ref["scalars"][t - 1], exact_k=True)
+        scale = float(res["next_scale"]) if wl.dynamic else 1.0
+    for name, t_ in (("master", opt.master), ("m", opt.exp_avg), ("v", opt.exp_avg_sq)):
+        same = check_state(name, to_np(t_), ref[name], wl.world)
+        assert same == 1.0, (name, same)
+    d = half_ulp_distance(to_np(opt.params), ref["params"])
+    record("params", None, ref["params"], ulp=d)
+    assert d.max() == 0
+    if wl.dynamic:
+        assert [r["skipped"] for r in ref["scalars"]] == [0, 1, 0, 0]
+
+
+def test_step_resident_refusals():
+    opt = zb.ZeroOptimizer([(10000,)], 4, 3000)
+    g = [torch.zeros(opt.plan.n_pad, dtype=torch.bfloat16, device="cuda")] * 4
+    with pytest.raises(zb.ZeroError) as e:
+        opt.step_resident(g)
+    assert e.value.code == zb.ZERO_EINVAL and "world_size <= 2" in e.value.message
+    opt = zb.ZeroOptimizer([(10000,)], 2, 3000)
+    g = [torch.zeros(opt.plan.n_pad, dtype=torch.bfloat16, device="cuda")] * 2
+    opt.reduce_scatter_bucket(0, g)
+    with pytest.raises(zb.ZeroError) as e:
+        opt.step_resident(g)
+    assert e.value.code == zb.ZERO_ESTATE

@@ -514,6 +514,59 @@ int zero_step(zero_plan* plan, const zero_adamw_cfg* cfg, float* master, float* 
                           workspace, stream);
 }
 
+int zero_step_resident(zero_plan* plan, const zero_adamw_cfg* cfg, int32_t grad_dtype,
+                       const void* const* replica_grads, float* master, float* exp_avg,
+                       float* exp_avg_sq, void* params, int32_t param_dtype, void* workspace,
+                       void* stream) {
+  NvtxRange nvtx("zero_step_resident");
+  if (!plan || !workspace) return fail(ZERO_EINVAL, "NULL argument");
+  if (int rc = check_dtype(grad_dtype, "zero_step_resident")) return rc;
+  if (int rc = check_dtype(param_dtype, "zero_step_resident")) return rc;
+  if (int rc = check_adamw(cfg)) return rc;
+  if (plan->world > 2)
+    return fail(ZERO_EINVAL,
+                "zero_step_resident moves fewer bytes only for world_size <= 2; use "
+                "zero_reduce_scatter_bucket and zero_step");
+  if (plan->n_pad > 0 && (!master || !exp_avg || !exp_avg_sq || !params || !replica_grads))
+    return fail(ZERO_EINVAL, "NULL argument");
+  if (!aligned16(workspace) || (plan->n_pad > 0 && (!aligned16(master) || !aligned16(exp_avg) ||
+                                                    !aligned16(exp_avg_sq) || !aligned16(params))))
+    return fail(ZERO_EALIGN, "step buffers and workspace must be 16-byte aligned");
+  if (plan->reduced_count != 0 || plan->n_micro != 0)
+    return fail(ZERO_ESTATE, "zero_step_resident after buckets of this step were already reduced");
+  const uint16_t* g[ZERO_MAX_WORLD];
+  for (int r = 0; r < plan->world && plan->n_pad > 0; ++r) {
+    if (!replica_grads[r]) return fail(ZERO_EINVAL, "replica_grads[" + std::to_string(r) + "] is NULL");
+    if (!aligned16(replica_grads[r]))
+      return fail(ZERO_EALIGN, "replica_grads[" + std::to_string(r) + "] is not 16-byte aligned");
+    g[r] = (const uint16_t*)replica_grads[r];
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  // the sum of squares of every bucket; the reduced gradient is not stored
+  for (int64_t b = 0; b < plan->n_buckets; ++b) {
+    const int64_t start = b * plan->bucket, len = bucket_len(plan, b);
+    const uint16_t* gb[ZERO_MAX_WORLD];
+    for (int r = 0; r < plan->world; ++r) gb[r] = g[r] + start;
+    int grid = 1;
+    cudaError_t e = rs_grid(len, plan->world, grad_dtype, &grid);
+    if (e != cudaSuccess) return cuda_fail(e, "reduce-scatter occupancy query");
+    e = launch_reduce_scatter(plan->world, grad_dtype, gb, nullptr, len,
+                              ws_partial(plan, workspace) + b * plan->slots_full,
+                              ws_bucket_blocks(plan, workspace) + b,
+                              &((WsHeader*)workspace)->result.device_error, grid, s,
+                              /*accumulate=*/0, /*want_sumsq=*/1, /*store=*/0);
+    if (e != cudaSuccess) return cuda_fail(e, "sum-of-squares launch");
+  }
+  cudaError_t e = launch_finalize(workspace, ws_bucket_blocks(plan, workspace), plan->slots_full,
+                                  ws_partial(plan, workspace), plan->n_buckets, *cfg, s);
+  if (e != cudaSuccess) return cuda_fail(e, "finalize launch");
+  e = launch_update_resident(plan->world, grad_dtype, param_dtype, g, master, exp_avg,
+                             exp_avg_sq, params, plan->n_pad, workspace, s);
+  if (e != cudaSuccess) return cuda_fail(e, "update launch");
+  plan->finalized = false;
+  return ZERO_OK;
+}
+
 int zero_all_gather(const zero_plan* plan, const void* params, void* const* rank_params,
                     int32_t n_dst, int32_t param_dtype, void* stream) {
   if (!plan) return fail(ZERO_EINVAL, "NULL argument");

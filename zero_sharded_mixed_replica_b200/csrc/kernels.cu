@@ -235,6 +235,7 @@ struct RsArgs {
   int32_t* device_error;              // sticky error word, or null
   int32_t accumulate;                 // 1: R += this pass's sum (later micro-batches)
   int32_t want_sumsq;                 // 1: accumulate the sum of squares (last pass)
+  int32_t store;                      // 0: R is not written (only the sum of squares)
 };
 
 // Pipeline shape of the reduce-scatter: each of kRsStages shared-memory stages holds the
@@ -279,8 +280,10 @@ __device__ __forceinline__ void finish8(const RsArgs& a, float* R, float (&acc)[
     acc[7] = __fadd_rn(o1.w, acc[7]);
   }
   // R is read back only after every bucket of the step: stream it past the caches
-  st_cs_f4(R, acc[0], acc[1], acc[2], acc[3]);
-  st_cs_f4(R + 4, acc[4], acc[5], acc[6], acc[7]);
+  if (a.store) {
+    st_cs_f4(R, acc[0], acc[1], acc[2], acc[3]);
+    st_cs_f4(R + 4, acc[4], acc[5], acc[6], acc[7]);
+  }
   if (a.want_sumsq) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -387,7 +390,7 @@ __global__ void __launch_bounds__(kRsTmaThreads, 1)
 #pragma unroll
         for (int r = 1; r < W; ++r) acc = __fadd_rn(acc, half_bits_to_float<DT>(a.g[r][i]));
         if (a.accumulate) acc = __fadd_rn(a.R[i], acc);
-        a.R[i] = acc;
+        if (a.store) a.R[i] = acc;
         if (a.want_sumsq) {
           const double d = (double)acc;
           ss = __fma_rn(d, d, ss);
@@ -704,6 +707,162 @@ __global__ void __launch_bounds__(kUpTmaThreads, 1)
   }
 }
 
+// ================================================================== K3': resident replicas
+
+// AdamW + cast for a step whose W replica gradients are still resident when the update
+// runs (worth it for W <= 2): the reduced gradient of every element is formed again from
+// the replica tiles -- the same rank-ordered fp32 sum as the bucket kernel, so the same
+// bits -- instead of being stored by the bucket kernel and read back. A step then moves
+// 4W + 26 bytes per parameter instead of 2W + 34. Pipeline as K3; a stage holds the W
+// replica tiles (halves) and the p, m, v tiles (fp32) of kUpTile elements.
+constexpr int kResMaxWorld = 2;
+struct UpResArgs {
+  const uint16_t* g[kResMaxWorld];  // replica r, element 0 of the flat space
+  float* p;
+  float* m;
+  float* v;
+  uint16_t* out;  // the gathered half buffer
+  int64_t n;
+  const WsHeader* h;
+  int32_t* device_error;
+};
+
+template <int W>
+__host__ __device__ constexpr size_t up_res_stage_bytes() {
+  return (size_t)kUpTile * (W * sizeof(uint16_t) + 3 * sizeof(float));
+}
+template <int W>
+__host__ __device__ constexpr size_t up_res_smem_bytes() {
+  return kUpStages * up_res_stage_bytes<W>() + 2 * kUpStages * sizeof(uint64_t);
+}
+
+template <int GD>
+__device__ __forceinline__ void unpack4(const uint2& x, float (&f)[4]) {
+  unpack2<GD>(x.x, f[0], f[1]);
+  unpack2<GD>(x.y, f[2], f[3]);
+}
+
+template <int W, int GD, int PD>
+__global__ void __launch_bounds__(kUpTmaThreads, 1)
+    adamw_resident_kernel(const __grid_constant__ UpResArgs a) {
+  constexpr size_t kStage = up_res_stage_bytes<W>();
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t* full = (uint64_t*)(smem + kUpStages * kStage);
+  uint64_t* empty = full + kUpStages;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    for (int st = 0; st < kUpStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], kUpConsumers / 32);
+    }
+    mbar_init_fence();
+  }
+  __syncthreads();
+  pdl_launch_dependents();
+  pdl_wait();
+
+  const WsHeader* h = a.h;
+  if (h->skip) return;  // overflow: the whole step is skipped (every thread)
+  AdamConsts c;
+  c.k = h->k;
+  c.b1 = h->b1;
+  c.omb1 = h->omb1;
+  c.b2 = h->b2;
+  c.omb2 = h->omb2;
+  c.bc1 = h->bc1;
+  c.bc2 = h->bc2;
+  c.eps = h->eps;
+  c.lr = h->lr;
+  c.decay = h->decay;
+
+  const int64_t n_tiles = a.n / kUpTile;
+  const int64_t G = gridDim.x;
+
+  if (tid >= kUpConsumers) {
+    if (tid == kUpConsumers) {  // producer
+      int64_t k = 0;
+      for (int64_t t = blockIdx.x; t < n_tiles; t += G, ++k) {
+        const int st = (int)(k % kUpStages);
+        if (k >= kUpStages &&
+            !mbar_wait(&empty[st], (uint32_t)((k / kUpStages - 1) & 1))) {
+          atomicOr(a.device_error, 1);
+          break;
+        }
+        if (*(volatile int32_t*)a.device_error) break;
+        mbar_arrive_expect_tx(&full[st], (uint32_t)kStage);
+        const int64_t off = t * kUpTile;
+        unsigned char* dst = smem + st * kStage;
+#pragma unroll
+        for (int r = 0; r < W; ++r)
+          bulk_load(dst + (size_t)r * kUpTile * sizeof(uint16_t), a.g[r] + off,
+                    kUpTile * sizeof(uint16_t), &full[st]);
+        float* f = (float*)(dst + (size_t)W * kUpTile * sizeof(uint16_t));
+        bulk_load(f, a.p + off, kUpTile * 4, &full[st]);
+        bulk_load(f + kUpTile, a.m + off, kUpTile * 4, &full[st]);
+        bulk_load(f + 2 * kUpTile, a.v + off, kUpTile * 4, &full[st]);
+      }
+      for (int64_t j = k > kUpStages ? k - kUpStages : 0; j < k; ++j)
+        if (!mbar_wait(&full[j % kUpStages], (uint32_t)((j / kUpStages) & 1)))
+          atomicOr(a.device_error, 4);
+    }
+    return;
+  }
+
+  int64_t k = 0;
+  for (int64_t t = blockIdx.x; t < n_tiles; t += G, ++k) {
+    const int st = (int)(k % kUpStages);
+    if (!mbar_wait(&full[st], (uint32_t)((k / kUpStages) & 1))) {
+      atomicOr(a.device_error, 2);
+      break;
+    }
+    const unsigned char* base = smem + st * kStage;
+    const uint16_t* gs = (const uint16_t*)base;
+    const float* fs = (const float*)(base + (size_t)W * kUpTile * sizeof(uint16_t));
+    const int64_t off = t * kUpTile;
+#pragma unroll
+    for (int q = 0; q < kUpTile / (4 * kUpConsumers); ++q) {
+      const int e = (q * kUpConsumers + tid) * 4;
+      float r[4];
+      unpack4<GD>(*(const uint2*)(gs + e), r);
+#pragma unroll
+      for (int w = 1; w < W; ++w) {
+        float x[4];
+        unpack4<GD>(*(const uint2*)(gs + w * kUpTile + e), x);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) r[j] = __fadd_rn(r[j], x[j]);
+      }
+      float4 p = *(const float4*)(fs + e);
+      float4 m = *(const float4*)(fs + kUpTile + e);
+      float4 v = *(const float4*)(fs + 2 * kUpTile + e);
+      adamw1(c, r[0], p.x, m.x, v.x);
+      adamw1(c, r[1], p.y, m.y, v.y);
+      adamw1(c, r[2], p.z, m.z, v.z);
+      adamw1(c, r[3], p.w, m.w, v.w);
+      st_f4(a.p + off + e, p.x, p.y, p.z, p.w);
+      st_f4(a.m + off + e, m.x, m.y, m.z, m.w);
+      st_f4(a.v + off + e, v.x, v.y, v.z, v.w);
+      *(uint2*)(a.out + off + e) = make_uint2(pack2<PD>(p.x, p.y), pack2<PD>(p.z, p.w));
+    }
+    __syncwarp();
+    if ((tid & 31) == 0) mbar_arrive(&empty[st]);
+  }
+
+  // the ragged tail after the last full tile
+  if (blockIdx.x == G - 1) {
+    for (int64_t i = n_tiles * kUpTile + tid; i < a.n; i += kUpConsumers) {
+      float r = half_bits_to_float<GD>(a.g[0][i]);
+#pragma unroll
+      for (int w = 1; w < W; ++w) r = __fadd_rn(r, half_bits_to_float<GD>(a.g[w][i]));
+      float p = a.p[i], m = a.m[i], v = a.v[i];
+      adamw1(c, r, p, m, v);
+      a.p[i] = p;
+      a.m[i] = m;
+      a.v[i] = v;
+      a.out[i] = (uint16_t)float_to_half_bits<PD>(p);
+    }
+  }
+}
+
 // ================================================================== small kernels
 
 template <int DT>
@@ -955,11 +1114,12 @@ cudaError_t launch_state_write(void* ws, const zero_scaler_state& st, cudaStream
 cudaError_t launch_reduce_scatter(int world, int dtype, const uint16_t* const* g, float* R,
                                   int64_t len, double* partial, int32_t* bucket_blocks,
                                   int32_t* device_error, int grid, cudaStream_t s,
-                                  int accumulate, int want_sumsq) {
+                                  int accumulate, int want_sumsq, int store) {
   RsArgs a;
   a.device_error = device_error;
   a.accumulate = accumulate;
   a.want_sumsq = want_sumsq;
+  a.store = store;
   for (int r = 0; r < ZERO_MAX_WORLD; ++r) a.g[r] = r < world ? g[r] : nullptr;
   a.R = R;
   a.partial = partial;
@@ -1056,6 +1216,45 @@ cudaError_t launch_update(int dtype, const float* R, float* master, float* m, fl
   if (grid < 1) grid = 1;
   void* args[] = {&a};
   return launch_chained(k, dim3((unsigned)grid), dim3(kUpTmaThreads), args, kUpSmemBytes, s);
+}
+
+cudaError_t launch_update_resident(int world, int gdt, int pdt, const uint16_t* const* g,
+                                   float* master, float* m, float* v, void* params, int64_t n,
+                                   const void* ws, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  WsHeader* h = (WsHeader*)ws;
+  UpResArgs a;
+  for (int r = 0; r < kResMaxWorld; ++r) a.g[r] = r < world ? g[r] : nullptr;
+  a.p = master;
+  a.m = m;
+  a.v = v;
+  a.out = (uint16_t*)params;
+  a.n = n;
+  a.h = h;
+  a.device_error = &h->result.device_error;
+  const void* table[2][2][2] = {
+      {{(const void*)adamw_resident_kernel<1, ZERO_BF16, ZERO_BF16>,
+        (const void*)adamw_resident_kernel<1, ZERO_BF16, ZERO_FP16>},
+       {(const void*)adamw_resident_kernel<1, ZERO_FP16, ZERO_BF16>,
+        (const void*)adamw_resident_kernel<1, ZERO_FP16, ZERO_FP16>}},
+      {{(const void*)adamw_resident_kernel<2, ZERO_BF16, ZERO_BF16>,
+        (const void*)adamw_resident_kernel<2, ZERO_BF16, ZERO_FP16>},
+       {(const void*)adamw_resident_kernel<2, ZERO_FP16, ZERO_BF16>,
+        (const void*)adamw_resident_kernel<2, ZERO_FP16, ZERO_FP16>}}};
+  const void* k = table[world - 1][gdt == ZERO_FP16][pdt == ZERO_FP16];
+  const size_t smem = world == 1 ? up_res_smem_bytes<1>() : up_res_smem_bytes<2>();
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kUpTmaThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  int64_t grid = (int64_t)per_sm * sm_count();
+  const int64_t n_tiles = n / kUpTile;
+  if (grid > n_tiles) grid = n_tiles;
+  if (grid < 1) grid = 1;
+  void* args[] = {&a};
+  return launch_chained(k, dim3((unsigned)grid), dim3(kUpTmaThreads), args, smem, s);
 }
 
 cudaError_t launch_cast(int dtype, const float* master, void* params, int64_t n,

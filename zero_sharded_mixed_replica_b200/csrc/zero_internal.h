@@ -96,7 +96,12 @@ cudaError_t launch_selftest_wait(void* ws, cudaStream_t s);
 cudaError_t launch_reduce_scatter(int world, int dtype, const uint16_t* const* g, float* R,
                                   int64_t len, double* partial, int32_t* bucket_blocks,
                                   int32_t* device_error, int grid, cudaStream_t s,
-                                  int accumulate = 0, int want_sumsq = 1);
+                                  int accumulate = 0, int want_sumsq = 1, int store = 1);
+// AdamW + cast with the reduced gradient formed again from W <= 2 resident replicas
+// (g[r]: replica r at flat element 0)
+cudaError_t launch_update_resident(int world, int gdt, int pdt, const uint16_t* const* g,
+                                   float* master, float* m, float* v, void* params, int64_t n,
+                                   const void* ws, cudaStream_t s);
 cudaError_t launch_finalize(void* ws, const int32_t* bucket_blocks, int64_t slots_full,
                             const double* partial, int64_t n_buckets,
                             const zero_adamw_cfg& cfg, cudaStream_t s);

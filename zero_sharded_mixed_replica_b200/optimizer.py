@@ -16,7 +16,8 @@ import torch
 from . import (AdamWCfg, Plan, ScalerCfg, adamw_cfg, scaler_cfg, zero_all_gather,
                zero_cast_params, zero_get_result, zero_reduce_scatter_bucket,
                zero_reduce_scatter_bucket_accum, zero_reduce_scatter_bucket_host,
-               zero_state_init, zero_step, zero_step_finalize, zero_step_update)
+               zero_state_init, zero_step, zero_step_finalize, zero_step_resident,
+               zero_step_update)
 
 _TORCH_HALF = {"bf16": torch.bfloat16, "fp16": torch.float16}
 
@@ -105,6 +106,15 @@ class ZeroOptimizer:
         for b in range(self.plan.n_buckets):
             self.reduce_scatter_bucket(b, replica_grads, base_offset)
         self.step()
+
+    def step_resident(self, replica_grads: Sequence) -> None:
+        """The whole step from whole-model replica buffers that stay resident, for
+        world_size <= 2: the update re-reads the replicas instead of a stored reduced
+        gradient (4W + 26 instead of 2W + 34 bytes per parameter); results are the same
+        bits as full_step. `reduced` is not written."""
+        zero_step_resident(self.plan, self.adamw, self.dtype, replica_grads, self._b("master"),
+                           self._b("exp_avg"), self._b("exp_avg_sq"), self._b("params"),
+                           self.dtype, self._b("workspace"), self._s())
 
     def overlapped_step(self, produce, slots: Sequence[Sequence], producer_stream) -> None:
         """One step whose reduce-scatter of bucket b overlaps the production of the next
