@@ -175,3 +175,22 @@ def test_binding_checks_tensor_arguments():
                                       b0, [3 << 20, 4 << 20], R, ws)
     ws_host = torch.zeros(p.workspace_bytes(), dtype=torch.uint8)
     assert "device memory" in _msg(zb.zero_state_init, p, ws_host, zb.scaler_cfg(False))
+
+
+def test_step_resident_refusals_before_any_device_work():
+    cfg = zb.adamw_cfg()
+    ws, m = 1 << 20, 2 << 20  # fake aligned device addresses, never dereferenced here
+    p4 = zb.Plan([(1024,)], 4, 512)
+    assert _code(zb.zero_step_resident, p4, cfg, "bf16", [m] * 4, m, m, m, m, "bf16", ws) \
+        == zb.ZERO_EINVAL  # world_size > 2
+    p2 = zb.Plan([(1024,)], 2, 512)
+    assert _code(zb.zero_step_resident, p2, cfg, 7, [m] * 2, m, m, m, m, "bf16", ws) \
+        == zb.ZERO_EINVAL  # grad dtype
+    assert _code(zb.zero_step_resident, p2, cfg, "bf16", [m, m + 2], m, m, m, m, "bf16", ws) \
+        == zb.ZERO_EALIGN
+    assert _code(zb.zero_step_resident, p2, cfg, "bf16", [m, 0], m, m, m, m, "bf16", ws) \
+        == zb.ZERO_EINVAL
+    assert _code(zb.zero_step_resident, p2, cfg, "bf16", [m] * 2, m + 4, m, m, m, "bf16", ws) \
+        == zb.ZERO_EALIGN
+    assert _code(zb.zero_step_resident, p2, zb.adamw_cfg(beta1=1.0), "bf16", [m] * 2, m, m, m,
+                 m, "bf16", ws) == zb.ZERO_EINVAL
