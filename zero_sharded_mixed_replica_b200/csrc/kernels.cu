@@ -1,9 +1,12 @@
 // kernels.cu -- sm_100a kernels of the ZeRO partitioned optimizer step.
 //
 // All kernels here are HBM-bandwidth bound streams (about 0.3 flop per byte); none is
-// a contraction, so none uses tensor cores. Each is a persistent grid-stride loop over
-// 16-byte vectors, sized from the SM count and the kernel's occupancy, with loads
-// marked L1::no_allocate (every byte is touched once per step).
+// a contraction, so none uses tensor cores. The step's kernels (bucket reduction,
+// update) and the all-gather copies are persistent grids of one CTA per SM fed by TMA:
+// a producer thread moves tiles between global and shared memory with 1-D bulk copies
+// through an mbarrier ring while the CTA's other threads compute from shared memory;
+// every wait is bounded. The small kernels (cast, state) are grid-stride loops over
+// 16-byte vectors. Every byte of a step is touched once, so nothing is kept in L1.
 //
 // Floating-point operations on the data path use the explicitly rounded intrinsics
 // (__fadd_rn, __fmul_rn, __fdiv_rn, __fsqrt_rn and the fp64 ones) so that the compiler

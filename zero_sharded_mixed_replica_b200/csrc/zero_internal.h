@@ -16,7 +16,7 @@ namespace zero {
 // elements, at most kRsMaxBlocks per bucket (a launch uses at most that many blocks).
 constexpr int kRsThreads = 256;
 constexpr int kRsMaxBlocks = 148 * 8;
-// Launch shape of the small grid-stride kernels (cast, replicate).
+// Launch shape of the small grid-stride kernels (cast).
 constexpr int kUpThreads = 256;
 constexpr int kFinalizeThreads = 1024;
 
