@@ -282,6 +282,17 @@ ZERO_API int zero_step_update(zero_plan* plan, float* master, float* exp_avg, fl
                      const float* reduced, void* params, int32_t param_dtype,
                      const void* workspace, void* stream);
 
+/* zero_step_full: the whole step in one call -- zero_reduce_scatter_bucket for every
+ * bucket in order, then zero_step -- for replica buffers that hold every bucket
+ * (replica_grads[r][i] is flat element i; replica_base_offset must be 0). Every argument
+ * is checked before the first launch, so a refused call changes nothing. Arguments and
+ * errors as for those calls; ESTATE when buckets of this step were already
+ * reduce-scattered. */
+ZERO_API int zero_step_full(zero_plan* plan, const zero_adamw_cfg* cfg, int32_t grad_dtype,
+                            const void* const* replica_grads, int64_t replica_base_offset,
+                            float* reduced, float* master, float* exp_avg, float* exp_avg_sq,
+                            void* params, int32_t param_dtype, void* workspace, void* stream);
+
 /* zero_step_resident: the whole step for W <= 2 ranks whose replica gradients are all
  * still in device memory when the step runs ([Z1] 2.1 the reduce-scatter of gradients
  * and the per-partition update; the schedule is this library's). The bucket kernel

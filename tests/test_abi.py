@@ -194,3 +194,18 @@ def test_step_resident_refusals_before_any_device_work():
         == zb.ZERO_EALIGN
     assert _code(zb.zero_step_resident, p2, zb.adamw_cfg(beta1=1.0), "bf16", [m] * 2, m, m, m,
                  m, "bf16", ws) == zb.ZERO_EINVAL
+
+
+def test_step_full_refusals_before_any_device_work():
+    cfg = zb.adamw_cfg()
+    ws, m = 1 << 20, 2 << 20  # fake aligned device addresses, never dereferenced here
+    p = zb.Plan([(1024,)], 2, 512)
+    call = zb.zero_step_full
+    assert _code(call, p, cfg, "bf16", [m] * 2, 5, m, m, m, m, m, "bf16", ws) == zb.ZERO_EINVAL
+    assert _code(call, p, cfg, 7, [m] * 2, 0, m, m, m, m, m, "bf16", ws) == zb.ZERO_EINVAL
+    assert _code(call, p, cfg, "bf16", [m, m + 2], 0, m, m, m, m, m, "bf16", ws) == zb.ZERO_EALIGN
+    assert _code(call, p, cfg, "bf16", [m, 0], 0, m, m, m, m, m, "bf16", ws) == zb.ZERO_EINVAL
+    assert _code(call, p, cfg, "bf16", [m] * 2, 0, m + 4, m, m, m, m, "bf16", ws) == zb.ZERO_EALIGN
+    assert _code(call, p, cfg, "bf16", [m] * 2, 0, None, m, m, m, m, "bf16", ws) == zb.ZERO_EINVAL
+    assert _code(call, p, zb.adamw_cfg(eps=0.0), "bf16", [m] * 2, 0, m, m, m, m, m, "bf16", ws) \
+        == zb.ZERO_EINVAL

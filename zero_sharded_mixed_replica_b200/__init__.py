@@ -142,6 +142,7 @@ def _load():
         "zero_step": [vp, P(AdamWCfg), vp, vp, vp, vp, vp, i32, vp, vp],
         "zero_step_finalize": [vp, P(AdamWCfg), vp, vp],
         "zero_step_resident": [vp, P(AdamWCfg), i32, vp, vp, vp, vp, vp, i32, vp, vp],
+        "zero_step_full": [vp, P(AdamWCfg), i32, vp, i64, vp, vp, vp, vp, vp, i32, vp, vp],
         "zero_step_update": [vp, vp, vp, vp, vp, vp, i32, vp, vp],
         "zero_all_gather": [vp, vp, vp, i32, i32, vp],
         "zero_get_result": [vp, P(StepResult), vp],
@@ -439,6 +440,23 @@ def zero_step(plan: Plan, cfg: AdamWCfg, master, exp_avg, exp_avg_sq, reduced, p
                          _buf(params, _dtype_name(param_dtype), n, "params"), _dtype(param_dtype),
                          _buf(workspace, "bytes", plan.workspace_bytes(), "workspace"),
                          _stream(stream)))
+
+
+def zero_step_full(plan: Plan, cfg: AdamWCfg, grad_dtype, replica_grads: Sequence,
+                   replica_base_offset: int, reduced, master, exp_avg, exp_avg_sq, params,
+                   param_dtype, workspace, stream=None) -> None:
+    n, gk = plan.n_pad, _dtype_name(grad_dtype)
+    need = max(0, n - int(replica_base_offset))
+    reps = (ctypes.c_void_p * len(replica_grads))(
+        *[_buf(g, gk, need, f"replica_grads[{r}]") for r, g in enumerate(replica_grads)])
+    _check(lib.zero_step_full(plan.handle, ctypes.byref(cfg), _dtype(grad_dtype), reps,
+                              int(replica_base_offset), _buf(reduced, "f32", n, "reduced"),
+                              _buf(master, "f32", n, "master"), _buf(exp_avg, "f32", n, "exp_avg"),
+                              _buf(exp_avg_sq, "f32", n, "exp_avg_sq"),
+                              _buf(params, _dtype_name(param_dtype), n, "params"),
+                              _dtype(param_dtype),
+                              _buf(workspace, "bytes", plan.workspace_bytes(), "workspace"),
+                              _stream(stream)))
 
 
 def zero_step_resident(plan: Plan, cfg: AdamWCfg, grad_dtype, replica_grads: Sequence, master,

@@ -514,6 +514,40 @@ int zero_step(zero_plan* plan, const zero_adamw_cfg* cfg, float* master, float* 
                           workspace, stream);
 }
 
+int zero_step_full(zero_plan* plan, const zero_adamw_cfg* cfg, int32_t grad_dtype,
+                   const void* const* replica_grads, int64_t replica_base_offset,
+                   float* reduced, float* master, float* exp_avg, float* exp_avg_sq,
+                   void* params, int32_t param_dtype, void* workspace, void* stream) {
+  NvtxRange nvtx("zero_step_full");
+  // every check before the first launch, so that a refused call changes nothing
+  if (!plan || !workspace) return fail(ZERO_EINVAL, "NULL argument");
+  if (int rc = check_dtype(grad_dtype, "zero_step_full")) return rc;
+  if (int rc = check_dtype(param_dtype, "zero_step_full")) return rc;
+  if (int rc = check_adamw(cfg)) return rc;
+  if (plan->n_pad > 0 && (!reduced || !master || !exp_avg || !exp_avg_sq || !params ||
+                          !replica_grads))
+    return fail(ZERO_EINVAL, "NULL argument");
+  if (!aligned16(workspace) ||
+      (plan->n_pad > 0 && (!aligned16(reduced) || !aligned16(master) || !aligned16(exp_avg) ||
+                           !aligned16(exp_avg_sq) || !aligned16(params))))
+    return fail(ZERO_EALIGN, "step buffers and workspace must be 16-byte aligned");
+  if (replica_base_offset != 0)
+    return fail(ZERO_EINVAL, "replica_base_offset must be 0: the replicas hold every bucket");
+  if (plan->reduced_count != 0 || plan->n_micro != 0)
+    return fail(ZERO_ESTATE, "zero_step_full after buckets of this step were already reduced");
+  for (int r = 0; r < plan->world && plan->n_pad > 0; ++r) {
+    if (!replica_grads[r]) return fail(ZERO_EINVAL, "replica_grads[" + std::to_string(r) + "] is NULL");
+    if (!aligned16(replica_grads[r]))
+      return fail(ZERO_EALIGN, "replica_grads[" + std::to_string(r) + "] is not 16-byte aligned");
+  }
+  for (int64_t b = 0; b < plan->n_buckets; ++b)
+    if (int rc = zero_reduce_scatter_bucket(plan, b, grad_dtype, replica_grads,
+                                            replica_base_offset, reduced, workspace, stream))
+      return rc;
+  return zero_step(plan, cfg, master, exp_avg, exp_avg_sq, reduced, params, param_dtype,
+                   workspace, stream);
+}
+
 int zero_step_resident(zero_plan* plan, const zero_adamw_cfg* cfg, int32_t grad_dtype,
                        const void* const* replica_grads, float* master, float* exp_avg,
                        float* exp_avg_sq, void* params, int32_t param_dtype, void* workspace,

@@ -16,8 +16,8 @@ import torch
 from . import (AdamWCfg, Plan, ScalerCfg, adamw_cfg, scaler_cfg, zero_all_gather,
                zero_cast_params, zero_get_result, zero_reduce_scatter_bucket,
                zero_reduce_scatter_bucket_accum, zero_reduce_scatter_bucket_host,
-               zero_state_init, zero_step, zero_step_finalize, zero_step_resident,
-               zero_step_update)
+               zero_state_init, zero_step, zero_step_finalize, zero_step_full,
+               zero_step_resident, zero_step_update)
 
 _TORCH_HALF = {"bf16": torch.bfloat16, "fp16": torch.float16}
 
@@ -102,10 +102,12 @@ class ZeroOptimizer:
 
     # -------------------------------------------------------------- whole step
     def full_step(self, replica_grads: Sequence, base_offset: int = 0) -> None:
-        """Reduce-scatter every bucket from whole-model replica buffers, then step."""
-        for b in range(self.plan.n_buckets):
-            self.reduce_scatter_bucket(b, replica_grads, base_offset)
-        self.step()
+        """Reduce-scatter every bucket from whole-model replica buffers, then step (one
+        library call)."""
+        zero_step_full(self.plan, self.adamw, self.dtype, replica_grads, base_offset,
+                       self._b("reduced"), self._b("master"), self._b("exp_avg"),
+                       self._b("exp_avg_sq"), self._b("params"), self.dtype,
+                       self._b("workspace"), self._s())
 
     def step_resident(self, replica_grads: Sequence) -> None:
         """The whole step from whole-model replica buffers that stay resident, for
