@@ -12,6 +12,9 @@
  *      writing the rounded half-precision parameters straight into the gathered
  *      buffer (the all-gather of step 5 costs nothing extra on one GPU).
  *   5. zero_all_gather: optional copies of the gathered buffer into per-rank buffers.
+ * zero_step_full does 1.-4. in one call; zero_step_resident does them for W <= 2 with
+ * fewer bytes when the replicas stay resident. One process per rank: the rank-local
+ * calls further down.
  *
  * Sources (web pages; titles and sections):
  *  [Z1] "ZeRO技术解析：大模型分布式训练的革命性突破" (ZeRO explained): 1.2.1-1.2.3 (the three
