@@ -553,8 +553,11 @@ class Zero3Schedule:
 def zero3_gather(plan: Plan, tensors: Sequence[int], partitions: Sequence, dst,
                  stream=None) -> None:
     arr = (ctypes.c_int32 * max(len(tensors), 1))(*tensors)
-    _check(lib.zero3_gather(plan.handle, arr, len(tensors), _ptr_array(partitions) if partitions else None,
-                            _addr(dst), _stream(stream)))
+    table = plan.tensor_table
+    need = 2 * sum(table[t][1] for t in tensors if 0 <= t < len(table))  # 2-byte elements
+    _check(lib.zero3_gather(plan.handle, arr, len(tensors),
+                            _ptr_array(partitions) if partitions else None,
+                            _buf(dst, "bytes", need, "dst"), _stream(stream)))
 
 
 def zero_abi_version() -> int:
