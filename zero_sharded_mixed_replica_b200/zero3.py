@@ -35,7 +35,8 @@ def run_forward(plan: Plan, schedule: Zero3Schedule, partitions: Sequence[int],
         if op == ZERO3_FETCH:
             sizes = [table[t][1] for t in ids]
             buf = torch.empty(sum(sizes), dtype=dtype, device=device)
-            zero3_gather(plan, ids, partitions, buf, s)
+            # sized here for exactly these tensors: passed by address, unchecked
+            zero3_gather(plan, ids, partitions, buf.data_ptr(), s)
             off = 0
             for t, n in zip(ids, sizes):
                 live[t] = (next_id, off)
