@@ -553,11 +553,13 @@ class Zero3Schedule:
 def zero3_gather(plan: Plan, tensors: Sequence[int], partitions: Sequence, dst,
                  stream=None) -> None:
     arr = (ctypes.c_int32 * max(len(tensors), 1))(*tensors)
-    table = plan.tensor_table
-    need = 2 * sum(table[t][1] for t in tensors if 0 <= t < len(table))  # 2-byte elements
+    if dst is not None and not isinstance(dst, int):  # a tensor: check its length
+        table = plan.tensor_table
+        need = 2 * sum(table[t][1] for t in tensors if 0 <= t < len(table))  # 2-byte elements
+        dst = _buf(dst, "bytes", need, "dst")
     _check(lib.zero3_gather(plan.handle, arr, len(tensors),
-                            _ptr_array(partitions) if partitions else None,
-                            _buf(dst, "bytes", need, "dst"), _stream(stream)))
+                            _ptr_array(partitions) if partitions else None, dst,
+                            _stream(stream)))
 
 
 def zero_abi_version() -> int:
