@@ -607,3 +607,49 @@ def test_step_resident_refusals():
     with pytest.raises(zb.ZeroError) as e:
         opt.step_resident(g)
     assert e.value.code == zb.ZERO_ESTATE
+
+
+@pytest.mark.parametrize("gdt,pdt", [("bf16", "fp16"), ("fp16", "bf16")])
+@pytest.mark.parametrize("resident", [False, True], ids=["stored_R", "resident"])
+def test_gradient_and_parameter_dtypes_differ(gdt, pdt, resident):
+    """Gradients in one half type, the gathered parameters in the other (the kernels'
+    mixed instantiations), three buckets and a ragged tail, 2 steps, against the
+    oracle's step with the same pair of types: bit-identical."""
+    codes = {"bf16": synthgen.BF16, "fp16": synthgen.FP16}
+    W, n, bucket = 2, 200003, 70000
+    plan = zb.Plan([(n,)], W, bucket, 1)
+    n_pad = plan.n_pad
+    master0 = synthgen.master_random_host(0, n_pad, 0, 0.02)
+    grads = [synthgen.grads_host(0, n_pad, 0, r, 1, 3e-2, 0.0, 1.0, codes[gdt]) for r in range(W)]
+    cfg_o, hp = oracle.scaler_cfg(False), oracle.hparams()
+    st = oracle.state_init(cfg_o)
+    R = np.zeros(n_pad, np.float32)
+    master, m, v = master0.copy(), np.zeros(n_pad, np.float32), np.zeros(n_pad, np.float32)
+    params = oracle.f32_to_half(master0, codes[pdt])
+    for _ in range(2):
+        oracle.step(grads, codes[gdt], bucket, R, master, m, v, params, codes[pdt], cfg_o, hp, st)
+
+    s = stream()
+    dev = dict(device="cuda")
+    g_d = [torch.from_numpy(g.view(np.int16)).cuda() for g in grads]
+    M = torch.from_numpy(master0).cuda()
+    Mm, Vv = torch.zeros(n_pad, **dev), torch.zeros(n_pad, **dev)
+    Rd = torch.zeros(n_pad, **dev)
+    P = torch.zeros(n_pad, dtype=torch.int16, **dev)
+    ws = torch.zeros(plan.workspace_bytes(), dtype=torch.uint8, **dev)
+    cfg = zb.adamw_cfg()
+    zb.zero_state_init(plan, ws, zb.scaler_cfg(False), s)
+    zb.zero_cast_params(plan, M, P, pdt, s)
+    for _ in range(2):
+        if resident:
+            zb.zero_step_resident(plan, cfg, gdt, g_d, M, Mm, Vv, P, pdt, ws, s)
+        else:
+            for b in range(plan.n_buckets):
+                zb.zero_reduce_scatter_bucket(plan, b, gdt, g_d, 0, Rd, ws, s)
+            zb.zero_step(plan, cfg, M, Mm, Vv, Rd, P, pdt, ws, s)
+    assert zb.zero_get_result(ws, s)["adam_t"] == 2
+    for got, want in ((M, master), (Mm, m), (Vv, v)):
+        assert np.array_equal(to_np(got).view(np.uint32), want.view(np.uint32))
+    assert np.array_equal(to_np(P).view(np.uint16), params)
+    if not resident:
+        assert np.array_equal(to_np(Rd).view(np.uint32), R.view(np.uint32))
