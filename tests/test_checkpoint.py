@@ -1,6 +1,7 @@
 """Sharded checkpoints: the shard files hold exactly the partitions, a corrupted shard
 is refused, a reload (same or another W) restores the unpadded flat state, and a run
 continued from a checkpoint equals the run without the interruption."""
+import json
 import os
 
 import numpy as np
@@ -77,3 +78,36 @@ def test_continued_run_equals_uninterrupted(tmp_path):
                       (params, full["params"])):
         assert np.array_equal(got, want)
     assert (st.scale, st.adam_t, st.iter) == (full["state"].scale, full["state"].adam_t, 4)
+
+
+def test_refuses_damaged_or_foreign_directories(tmp_path):
+    n, W = 5000, 4
+    pl = oracle.plan([n], W, 1000, 1)
+    rng = np.random.default_rng(3)
+    master, m, v = (rng.standard_normal(pl.n_pad).astype(np.float32) for _ in range(3))
+    fields = dict(shapes=[[n]], world_size=W, reduce_bucket_size=1000, align=1, n=pl.n,
+                  n_pad=pl.n_pad, p=pl.p, dtype="bf16", scaler_cfg={}, scaler_state={},
+                  adamw={})
+    d = tmp_path / "ck"
+    ck.save_flat(str(d), fields, master, m, v)
+    # a shard cut short is refused before anything is read from it
+    shard = d / "rank00002.bin"
+    data = shard.read_bytes()
+    shard.write_bytes(data[:-4])
+    with pytest.raises(ValueError, match="bytes, expected"):
+        ck.load_flat(str(d))
+    shard.write_bytes(data)
+    assert np.array_equal(ck.load_flat(str(d))[1], master[:n])
+    # zeroed shard: refused by its checksum, read as it is without verification
+    shard.write_bytes(bytes(len(data)))
+    with pytest.raises(ValueError, match="checksum"):
+        ck.load_flat(str(d))
+    got = ck.load_flat(str(d), verify=False)[1]
+    lo, hi = 2 * pl.p, min(3 * pl.p, n)
+    assert not got[lo:hi].any() and np.array_equal(got[:lo], master[:lo])
+    # not a checkpoint of this format
+    meta = json.loads((d / "meta.json").read_text())
+    meta["format"] = "something-else"
+    (d / "meta.json").write_text(json.dumps(meta))
+    with pytest.raises(ValueError, match="not a"):
+        ck.load_flat(str(d))
