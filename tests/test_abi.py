@@ -209,3 +209,28 @@ def test_step_full_refusals_before_any_device_work():
     assert _code(call, p, cfg, "bf16", [m] * 2, 0, None, m, m, m, m, "bf16", ws) == zb.ZERO_EINVAL
     assert _code(call, p, zb.adamw_cfg(eps=0.0), "bf16", [m] * 2, 0, m, m, m, m, m, "bf16", ws) \
         == zb.ZERO_EINVAL
+
+
+@pytest.mark.parametrize("std", ["c99", "c11"])
+def test_header_compiles_as_plain_c(tmp_path, std):
+    """include/zero_b200.h is a C header: a C program that includes it and calls into
+    the library compiles without warnings under -pedantic."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use.c"
+    src.write_text('#include "zero_b200.h"\n'
+                   "int main(void) {\n"
+                   "  zero_plan* plan = 0;\n"
+                   "  const int64_t dims[1] = {1024};\n"
+                   "  const int32_t ndims[1] = {1};\n"
+                   "  int rc = zero_plan_create(dims, ndims, 1, 2, 512, 128, &plan);\n"
+                   "  if (rc == ZERO_OK) zero_plan_destroy(plan);\n"
+                   "  return zero_abi_version() == ZERO_ABI_VERSION ? rc : 1;\n"
+                   "}\n")
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    r = subprocess.run([cc, f"-std={std}", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                        "-fsyntax-only", "-I", inc, str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
