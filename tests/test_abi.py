@@ -213,8 +213,8 @@ def test_step_full_refusals_before_any_device_work():
 
 @pytest.mark.parametrize("std", ["c99", "c11"])
 def test_header_compiles_as_plain_c(tmp_path, std):
-    """include/zero_b200.h is a C header: a C program that includes it and calls into
-    the library compiles without warnings under -pedantic."""
+    """include/zero_b200.h is a C header: a C program that includes it, links against
+    libzero_b200.so and plans a step compiles without warnings under -pedantic and runs."""
     import shutil
     import subprocess
     cc = shutil.which("gcc") or shutil.which("cc")
@@ -230,7 +230,13 @@ def test_header_compiles_as_plain_c(tmp_path, std):
                    "  if (rc == ZERO_OK) zero_plan_destroy(plan);\n"
                    "  return zero_abi_version() == ZERO_ABI_VERSION ? rc : 1;\n"
                    "}\n")
-    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(zb.LIB_PATH)
+    exe = tmp_path / "use"
     r = subprocess.run([cc, f"-std={std}", "-Wall", "-Wextra", "-Werror", "-pedantic",
-                        "-fsyntax-only", "-I", inc, str(src)], capture_output=True, text=True)
+                        "-I", os.path.join(root, "include"), str(src), "-o", str(exe),
+                        "-L", libdir, "-lzero_b200", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+    # planning needs no GPU: the program runs here too
+    assert subprocess.run([str(exe)]).returncode == 0
